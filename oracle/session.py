@@ -1,0 +1,99 @@
+"""Whole-step oracle: window KV assembly, pooling, RoPE and attention in fp64.
+
+TEST INFRASTRUCTURE ONLY (see ``oracle/__init__.py``).
+
+The step follows the pages' order: the history tiers are pooled from the
+full-resolution frames (pre-RoPE K and V, pooled per head), every token of the
+window is placed at its window-relative position, Q and K are rotated, and
+each chunk query attends over all valid prompt, context and chunk keys with
+scale 1/sqrt(D).  Readings are listed in ``oracle/layout.py`` and below.
+
+Reading on what is pooled: the to_k / to_v projections are linear ("MiniMax-H3
+deep dive", tensor-name paragraph), so averaging latent tokens before the
+projection equals averaging K and V after it; the oracle averages K and V.
+"""
+from __future__ import annotations
+
+from typing import Dict, List, Optional, Sequence
+
+import numpy as np
+
+from . import attention, layout, pool, rope3d, _f64
+
+
+def pooled_tier(spec, frames_k, frames_v, ph: int, pw: int):
+    """Pool full-resolution frames [F x (Gh*Gw, H, D)] -> (K, V) [F*cells, H, D]
+    and positions of the cells relative to each frame ((mean row, mean col))."""
+    H, D = spec.n_heads, spec.head_dim
+    F = len(frames_k)
+    xk = np.stack([_f64(f) for f in frames_k]).reshape(F, spec.grid_h, spec.grid_w, H, D)
+    xv = np.stack([_f64(f) for f in frames_v]).reshape(F, spec.grid_h, spec.grid_w, H, D)
+    pk = pool(xk, ph, pw)
+    pv = pool(xv, ph, pw)
+    cells = pk.shape[1] * pk.shape[2]
+    return pk.reshape(F * cells, H, D), pv.reshape(F * cells, H, D)
+
+
+def session_kv(spec, inp) -> List[Dict]:
+    """Segments in buffer order: dicts with name, k (pre-RoPE), v [n, H, D] fp64
+    and pos [n, 3] fp64."""
+    H, D = spec.n_heads, spec.head_dim
+    segs = {name: {"name": name, "k": [], "v": [], "pos": []} for name in layout.segment_names(spec)}
+    segs["prompt"]["k"].append(_f64(inp.prompt_k))
+    segs["prompt"]["v"].append(_f64(inp.prompt_v))
+    segs["prompt"]["pos"] += [(0.0, 0.0, 0.0)] * spec.prompt_len
+    for f, (t, role, ph, pw, n) in enumerate(layout.context_plan(spec)):
+        s = segs[role]
+        if role.startswith("tier"):
+            k, v = pooled_tier(spec, [inp.ctx_k[f]], [inp.ctx_v[f]], ph, pw)
+            s["k"].append(k)
+            s["v"].append(v)
+            s["pos"] += [(t, mr, mc) for (_, _, _, _, mr, mc) in
+                         layout.pooled_cells(spec.grid_h, spec.grid_w, ph, pw)]
+        else:
+            s["k"].append(_f64(inp.ctx_k[f]))
+            s["v"].append(_f64(inp.ctx_v[f]))
+            for i in range(n):
+                r, c = layout.frame_token_rc(i, spec.grid_w)
+                s["pos"].append((t, float(r), float(c)))
+    segs["chunk"]["k"].append(_f64(inp.k))
+    segs["chunk"]["v"].append(_f64(inp.v))
+    segs["chunk"]["pos"] += layout.chunk_positions(spec)
+    out = []
+    for name in layout.segment_names(spec):
+        s = segs[name]
+        k = np.concatenate(s["k"]) if s["k"] else np.zeros((0, H, D))
+        v = np.concatenate(s["v"]) if s["v"] else np.zeros((0, H, D))
+        pos = np.asarray(s["pos"], dtype=np.float64).reshape(-1, 3)
+        assert k.shape[0] == v.shape[0] == pos.shape[0]
+        out.append({"name": name, "k": k, "v": v, "pos": pos})
+    return out
+
+
+def session_reference(spec, inp, heads: Optional[Sequence[int]] = None,
+                      rows: Optional[Sequence[int]] = None):
+    """O [n_rows, n_heads_sel, D] and LSE [n_rows, n_heads_sel] in fp64 for the
+    chunk queries ``rows`` (default all) and ``heads`` (default all)."""
+    H, D = spec.n_heads, spec.head_dim
+    heads = list(range(H)) if heads is None else list(heads)
+    segs = session_kv(spec, inp)
+    k_all = np.concatenate([s["k"][:, heads] for s in segs])
+    v_all = np.concatenate([s["v"][:, heads] for s in segs])
+    p_all = np.concatenate([s["pos"] for s in segs])
+    k_rot = rope3d(k_all, p_all, spec.rope_split, spec.rope_base)
+    q = _f64(inp.q)[:, heads]
+    q_pos = np.asarray(layout.chunk_positions(spec), dtype=np.float64)
+    if rows is not None:
+        rows = list(rows)
+        q = q[rows]
+        q_pos = q_pos[rows]
+    q_rot = rope3d(q, q_pos, spec.rope_split, spec.rope_base)
+    scale = 1.0 / np.sqrt(D)
+    n = q_rot.shape[0]
+    o = np.empty((n, len(heads), D))
+    lse = np.empty((n, len(heads)))
+    for hi in range(len(heads)):
+        o[:, hi], lse[:, hi] = attention(np.ascontiguousarray(q_rot[:, hi]),
+                                         np.ascontiguousarray(k_rot[:, hi]),
+                                         np.ascontiguousarray(v_all[:, hi]), scale)
+    return o, lse

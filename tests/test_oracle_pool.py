@@ -1,0 +1,126 @@
+"""Pins for the oracle's history-tier pooling and its window layout (CPU only)."""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import layout
+import workloads
+
+
+def _torch_avg_pool(x, ph, pw):
+    """Library reference: torch avg_pool2d, ceil mode, padding excluded from
+    the count.  x: [F, Gh, Gw, C] float64."""
+    t = torch.from_numpy(np.ascontiguousarray(x.transpose(0, 3, 1, 2)))
+    y = torch.nn.functional.avg_pool2d(t, (ph, pw), stride=(ph, pw), ceil_mode=True,
+                                       count_include_pad=False)
+    return y.numpy().transpose(0, 2, 3, 1)
+
+
+@pytest.mark.parametrize("grid,pool", [((5, 7), (2, 2)), ((5, 7), (4, 4)), ((24, 42), (2, 2)),
+                                       ((24, 42), (4, 4)), ((12, 21), (2, 2)), ((6, 8), (3, 2))])
+def test_pool_matches_torch_avg_pool(grid, pool):
+    x = np.random.default_rng(1).standard_normal((3,) + grid + (5,))
+    np.testing.assert_allclose(oracle.pool(x, *pool), _torch_avg_pool(x, *pool), rtol=0, atol=1e-14)
+
+
+def test_pool_brute_force_tiny():
+    Gh, Gw, ph, pw = 5, 7, 4, 4
+    x = np.random.default_rng(2).standard_normal((1, Gh, Gw, 1))
+    y = oracle.pool(x, ph, pw)
+    assert y.shape == (1, 2, 2, 1)
+    # cells by hand: rows {0..3},{4}; cols {0..3},{4..6}
+    np.testing.assert_allclose(y[0, 0, 0, 0], x[0, 0:4, 0:4, 0].mean(), atol=1e-15)
+    np.testing.assert_allclose(y[0, 0, 1, 0], x[0, 0:4, 4:7, 0].sum() / 12.0, atol=1e-15)
+    np.testing.assert_allclose(y[0, 1, 0, 0], x[0, 4, 0:4, 0].sum() / 4.0, atol=1e-15)
+    np.testing.assert_allclose(y[0, 1, 1, 0], x[0, 4, 4:7, 0].sum() / 3.0, atol=1e-15)
+
+
+def test_pool_constant_and_mass():
+    x = np.full((2, 24, 42, 3), 1.75)
+    assert np.all(oracle.pool(x, 4, 4) == 1.75)
+    x = np.random.default_rng(3).standard_normal((2, 24, 42, 3))
+    y = oracle.pool(x, 4, 4)
+    counts = np.array([[(r1 - r0) * (c1 - c0) for (r0, r1, c0, c1, _, _) in layout.pooled_cells(24, 42, 4, 4)]])
+    mass = (y.reshape(2, -1, 3) * counts.reshape(1, -1, 1)).sum(axis=1)
+    np.testing.assert_allclose(mass, x.sum(axis=(1, 2)), rtol=1e-13)
+
+
+def test_two_stage_equals_direct_on_divisible_grid():
+    """24x42 -> 2x2 -> 2x2 equals 4x4 (ceil) directly: T2 cells are all full."""
+    x = np.random.default_rng(4).standard_normal((2, 24, 42, 4))
+    np.testing.assert_allclose(oracle.pool(oracle.pool(x, 2, 2), 2, 2), oracle.pool(x, 4, 4), atol=1e-14)
+
+
+def test_pooled_cell_centroids_match_avg_pool_of_coordinates():
+    for (Gh, Gw, ph, pw) in [(24, 42, 4, 4), (24, 42, 2, 2), (5, 7, 4, 4)]:
+        rr, cc = np.meshgrid(np.arange(Gh, dtype=float), np.arange(Gw, dtype=float), indexing="ij")
+        ref = _torch_avg_pool(np.stack([rr, cc], -1)[None], ph, pw)[0].reshape(-1, 2)
+        got = np.array([(mr, mc) for (_, _, _, _, mr, mc) in layout.pooled_cells(Gh, Gw, ph, pw)])
+        assert np.array_equal(got, ref)
+
+
+def test_latent_geometry_from_pages(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "latent_geometry.json")))
+    s = g["vae_spatial_compression"] * g["dit_patch_thw"][1]
+    assert g["frame_width_px"] // s == workloads.GRID_W_FULL == 42
+    assert g["frame_height_px"] // s == workloads.GRID_H_FULL == 24
+    assert g["audio_sample_rate_hz"] / g["audio_hop"] == workloads.AUDIO_RATE == 40.0
+    assert g["video_fps"] / g["vae_temporal_compression"] == workloads.LATENT_FPS == 6.0
+    assert workloads.CHUNK.head_dim == g["head_dim"]
+
+
+def test_segment_lengths_and_capacities():
+    # tiered chunk: sink 1008, 12 frames x (6 x 11) cells, 9 frames x (12 x 21), 3 x 1008, 3 x 1008 + 20
+    sp = workloads.CHUNK_TIERED
+    assert layout.segment_names(sp) == ["prompt", "sink", "tier0", "tier1", "recent", "chunk"]
+    assert layout.segment_lengths(sp) == [256, 1008, 12 * 66, 9 * 252, 3024, 3044]
+    assert layout.capacities([sp]) == [256, 1024, 896, 2304, 3072, 3072]
+    assert layout.segment_offsets(layout.capacities([sp])) == [0, 256, 1280, 2176, 4480, 7552]
+    sp = workloads.CHUNK
+    assert layout.segment_lengths(sp) == [256, 1008, 3024, 3044]
+    sp = workloads.CLIP
+    assert layout.segment_names(sp) == ["prompt", "chunk"]
+    assert layout.segment_lengths(sp) == [256, 30440]
+    sp = workloads.TINY
+    assert layout.segment_lengths(sp) == [16, 48, 48, 100]
+
+
+def test_positions():
+    sp = workloads.CHUNK
+    pos = layout.chunk_positions(sp)
+    assert len(pos) == 3044
+    assert pos[0] == (0.0, 0.0, 0.0) and pos[1] == (0.0, 0.0, 1.0) and pos[42] == (0.0, 1.0, 0.0)
+    assert pos[3023] == (2.0, 23.0, 41.0)
+    assert pos[3024] == (0.0, 0.0, 0.0)
+    # audio i at i * 6 / 40 latent frames: token 20 would sit 0.5 s = 3 latent frames later
+    np.testing.assert_allclose([p[0] for p in pos[3024:]], np.arange(20) * 0.15, rtol=0, atol=1e-15)
+    plan = layout.context_plan(sp)
+    assert [p[0] for p in plan] == [-4.0, -3.0, -2.0, -1.0]
+    assert [p[1] for p in plan] == ["sink", "recent", "recent", "recent"]
+    plan = layout.context_plan(workloads.CHUNK_TIERED)
+    assert plan[0][:2] == (-25.0, "sink")
+    assert [p[1] for p in plan[1:13]] == ["tier0"] * 12 and plan[1][0] == -24.0 and plan[12][0] == -13.0
+    assert [p[1] for p in plan[13:22]] == ["tier1"] * 9 and plan[21][0] == -4.0
+    assert [p[1] for p in plan[22:]] == ["recent"] * 3
+
+
+def test_session_kv_places_input_tokens():
+    sp = workloads.scaled(workloads.CHUNK_TIERED, n_heads=2, head_dim=64, rope_split=(16, 24, 24),
+                          prompt_len=7, chunk_video_tokens=2 * 1008 + 5, chunk_audio_tokens=3)
+    inp = workloads.draw_session(sp, 11)
+    segs = oracle.session_kv(sp, inp)
+    by = {s["name"]: s for s in segs}
+    assert np.array_equal(by["prompt"]["k"], inp.prompt_k.double().numpy())
+    assert np.array_equal(by["sink"]["v"], inp.ctx_v[0].double().numpy())
+    assert np.array_equal(by["recent"]["k"], torch.cat(inp.ctx_k[22:]).double().numpy())
+    assert np.array_equal(by["chunk"]["v"], inp.v.double().numpy())
+    f = np.stack([t.double().numpy() for t in inp.ctx_k[1:13]]).reshape(12, 24, 42, -1)
+    ref = _torch_avg_pool(f, 4, 4).reshape(12 * 66, 2, 64)
+    np.testing.assert_allclose(by["tier0"]["k"], ref, atol=1e-14)
+    assert by["chunk"]["pos"][2 * 1008 + 4].tolist() == [2.0, 0.0, 4.0]
+    assert by["tier1"]["pos"][0].tolist() == [-12.0, 0.5, 0.5]
+    assert by["tier0"]["pos"][65].tolist() == [-24.0, 21.5, 40.5]
