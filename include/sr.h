@@ -1,0 +1,214 @@
+/*
+ * sr.h -- C ABI of libsr.so: the chunk-streaming joint video+audio
+ * self-attention step on one NVIDIA B200 (sm_100a).
+ *
+ * The step (one DiT layer, all heads) is four calls launched back to back on
+ * one CUDA stream:
+ *   sr_history_compress  pool history frames into coarser tiers
+ *   sr_kv_append         write token K/V (and positions) into the window
+ *   sr_rope3d_apply      3-D (t, h, w) RoPE + re-layout of Q and window K
+ *   sr_chunk_attention_fwd  softmax attention of the chunk queries over the
+ *                        prompt, context and chunk KV segments
+ *
+ * Conventions shared by every call
+ *   - Every function returns an int status (SR_OK or an SR_ERR_* code).  On
+ *     error nothing is launched and sr_get_last_error() (thread-local) holds
+ *     a one-line reason.
+ *   - Every tensor pointer is DEVICE memory owned by the caller.  The library
+ *     never allocates, frees or synchronises; launches are asynchronous on the
+ *     caller's stream (`stream` is a cudaStream_t passed as void*; NULL means
+ *     the legacy default stream).
+ *   - Tensors are bf16 unless stated; positions are fp32 triples (t, h, w).
+ *     Strides are in ELEMENTS.  The head dimension is contiguous (stride 1).
+ *     Pointers to bf16 tensors must be 16-byte aligned and every stride a
+ *     multiple of 8 elements (16 bytes); violations return SR_ERR_INVALID_ARG.
+ *   - Sizes are int32/int64 counts; a call with zero work returns SR_OK and
+ *     launches nothing.
+ */
+#ifndef SR_H_
+#define SR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SR_VERSION 1
+
+#define SR_OK 0
+#define SR_ERR_INVALID_ARG 1
+#define SR_ERR_UNSUPPORTED 2
+#define SR_ERR_CUDA 3
+#define SR_ERR_DEVICE_TIMEOUT 4
+
+#define SR_MAX_SEG 8   /* KV segments per window */
+#define SR_TILE 128    /* KV tile (tokens); every segment capacity is a multiple */
+
+/* Library version (SR_VERSION of the build). */
+int sr_version(void);
+
+/* Reason for the last non-OK status returned on this thread ("" if none). */
+const char *sr_get_last_error(void);
+
+/* ------------------------------------------------------------------------ */
+/* 3-D multimodal RoPE.
+ *
+ * Defined by: "MiniMax-H3 deep dive" (fiv.co.kr), H3-Omni-Transformer row of
+ * the components table and the tensor-name paragraph (3D MM-RoPE on the
+ * shared single-stream attention); the fused rotate-and-write-cache idea is
+ * from "StreamRender-H3" (molayo1419.me), causal VAE section (qk-norm, RoPE
+ * and KV-cache write fused in one kernel).
+ *
+ * Reading (the pages give no formula): the head vector is split into
+ * contiguous sub-blocks [t: d_t | h: d_h | w: d_w]; inside the sub-block of
+ * axis a (width d_a) the interleaved pair (x[2j], x[2j+1]) turns
+ * counter-clockwise by phi = pos_a * base^(-2j/d_a).
+ *
+ *   y = out_scale * R(pos) x            (computed in fp32, stored bf16 RNE)
+ *
+ * x   element (b, n, h, d) at x + b*x_batch_stride + n*x_token_stride + h*x_head_stride + d
+ * y   element (b, n, h, d) at y + b*y_batch_stride + n*y_token_stride + h*y_head_stride + d
+ * pos fp32 (t, h, w) of token (b, n) at pos + b*pos_batch_stride + 3*n; NULL = all zero
+ *     (a pure re-layout, optionally scaled).
+ * n_valid_dev  optional int32[n_batch] on the device: tokens n >= n_valid[b]
+ *     are skipped (neither read nor written).  NULL = all n_tokens.
+ * Layouts: any strides, e.g. token-major [B, N, H, D] in, head-major
+ * [B, H, N, D] out (the attention layout).  x and y must not overlap.
+ * Requirements: head_dim in {64, 128}; d_t + d_h + d_w == head_dim, each even
+ * and a multiple of 8; n_heads >= 1.
+ */
+typedef struct {
+    float base;                 /* 10000 */
+    int32_t d_t, d_h, d_w;      /* sub-block widths */
+} sr_rope_cfg;
+
+int sr_rope3d_apply(const void *x, void *y, const float *pos,
+                    int32_t n_batch, int32_t n_tokens, int32_t n_heads, int32_t head_dim,
+                    const int32_t *n_valid_dev, sr_rope_cfg cfg, float out_scale,
+                    int64_t x_batch_stride, int64_t x_token_stride, int64_t x_head_stride,
+                    int64_t y_batch_stride, int64_t y_token_stride, int64_t y_head_stride,
+                    int64_t pos_batch_stride, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* History-tier pooling.
+ *
+ * Defined by: "AlayaRenderer-Flash" (aitrends.kr), key contributions and
+ * technical details: past history is kept in three tiers by temporal
+ * distance, recent at full resolution, older at progressively lower spatial
+ * resolution.
+ *
+ * Reading: per frame, cell (r, c) of a pool_h x pool_w ceil-mode pooling is
+ * the mean of the source tokens in rows [r*ph, min((r+1)*ph, Gh)) x cols
+ * [c*pw, min((c+1)*pw, Gw)), counting valid members only, for K and V
+ * separately and per head (fp32 accumulation, bf16 RNE result).  The pooled
+ * position is (frame_t[f], mean member row, mean member col).
+ *
+ * Source token (b, f, i = row*Gw + col, h, d) at
+ *   in + b*in_batch_stride + f*in_frame_stride + i*in_token_stride + h*in_head_stride + d
+ * Pooled token (b, f, j = r*ceil(Gw/pw) + c, h, d) at
+ *   out + b*out_batch_stride + f*out_frame_stride + j*out_token_stride + h*out_head_stride + d
+ * k_in/k_out or v_in/v_out may both be NULL (that tensor is skipped).
+ * frame_t   fp32 [n_batch][n_frames] (device) -- required when pos_out != NULL
+ * pos_out   fp32 (t, h, w) of pooled token (b, f, j) at
+ *           pos_out + b*pos_batch_stride + 3*(f*cells + j); NULL = not written
+ * slot_of_src int32 [n_frames*Gh*Gw] (device): slot_of_src[f*Gh*Gw + i] =
+ *           f*cells + (cell of i); the same for every batch; NULL = not written
+ * Input and output must not overlap.  head_dim in {64, 128};
+ * pool_h, pool_w in [1, 8].
+ */
+typedef struct {
+    int32_t grid_h, grid_w;     /* source token grid (rows, cols) per frame */
+    int32_t pool_h, pool_w;     /* pooling window = stride */
+} sr_pool_cfg;
+
+int sr_history_compress(const void *k_in, const void *v_in, void *k_out, void *v_out,
+                        int32_t n_batch, int32_t n_frames, int32_t n_heads, int32_t head_dim,
+                        sr_pool_cfg cfg,
+                        int64_t in_batch_stride, int64_t in_frame_stride,
+                        int64_t in_token_stride, int64_t in_head_stride,
+                        int64_t out_batch_stride, int64_t out_frame_stride,
+                        int64_t out_token_stride, int64_t out_head_stride,
+                        const float *frame_t, float *pos_out, int64_t pos_batch_stride,
+                        int32_t *slot_of_src, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* KV append into the persistent window buffer.
+ *
+ * Defined by: "StreamRender-H3" (molayo1419.me), inference acceleration
+ * section: a per-layer persistent KV buffer kept in the layout the attention
+ * kernel reads, with only the dynamic region updated in place (no
+ * reallocation, no relocation of history); streaming context section: only
+ * the recent history and the current chunk are recomputed.
+ *
+ * The window buffers are head-major [n_batch][n_heads][buf_tokens][head_dim]
+ * (contiguous) for K and V, and fp32 [n_batch][buf_tokens][3] for positions.
+ * Token n of the source lands in slot dst_token + n:
+ *   k_buf[b][h][dst_token + n][:] = k_src + b*src_batch_stride + n*src_token_stride + h*src_head_stride
+ * (likewise V and pos_src -> pos_buf; pos_src token stride 3, batch stride
+ * pos_src_batch_stride).  Bytes are copied exactly.
+ * Any of k_src / v_src / pos_src may be NULL (that buffer is left alone).
+ * n_valid_dev: optional int32[n_batch]; tokens n >= n_valid[b] are skipped.
+ * Requires dst_token + n_tokens <= buf_tokens; head_dim in {64, 128}.
+ */
+int sr_kv_append(void *k_buf, void *v_buf, float *pos_buf,
+                 int32_t n_batch, int32_t n_heads, int32_t head_dim, int32_t buf_tokens,
+                 int32_t dst_token,
+                 const void *k_src, const void *v_src, const float *pos_src,
+                 int32_t n_tokens, const int32_t *n_valid_dev,
+                 int64_t src_batch_stride, int64_t src_token_stride, int64_t src_head_stride,
+                 int64_t pos_src_batch_stride, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Fused chunk attention over [prompt | context | chunk] KV segments.
+ *
+ * Defined by: "StreamRender-H3" (molayo1419.me), streaming context section
+ * (the window is attended bidirectionally; the moving part sees the whole
+ * window) and inference acceleration section (FlashAttention on Blackwell
+ * tuned to the streaming shapes with one KV split; lengths and offsets reused
+ * without host-device synchronisation; persistent KV in the kernel's
+ * layout); "AlayaRenderer-Flash" (aitrends.kr), methodology (past chunks as
+ * clean tokens in self-attention; persistent style-prompt KV in every
+ * self-attention layer).
+ *
+ *   O[b, i, h] = sum_j softmax_j(softmax_scale * q_i . k_j) v_j
+ *   over every VALID slot j of every segment; LSE = ln sum_j exp(scale q.k_j)
+ *
+ * No causal mask.  Padded slots (beyond a segment's valid length) are masked.
+ *
+ * q    [n_batch][n_heads][q_cap][head_dim]      (head-major, after RoPE)
+ * k, v [n_batch][n_heads][kv_tokens][head_dim]  kv_tokens = sum(layout->cap)
+ *      segment s occupies slots [start_s, start_s + cap_s), start_s = sum_{t<s} cap_t;
+ *      its valid tokens are the first kv_len[b][s] slots.
+ *      Padded V slots must hold finite values (zero-fill the buffer once).
+ * o    [n_batch][q_cap][n_heads][head_dim]      (token-major, bf16)
+ * lse  fp32 [n_batch][n_heads][q_cap] natural-log LSE, or NULL
+ * kv_len_dev int32 [n_batch][layout->n_seg] (device), 0 <= len <= cap
+ * q_len_dev  int32 [n_batch] (device), 1 <= q_len <= q_cap; rows >= q_len are
+ *      neither computed into o nor lse.
+ * status_dev optional int32 (device): left untouched on success; set to
+ *      SR_ERR_DEVICE_TIMEOUT if a pipeline wait inside the kernel gave up
+ *      (bounded waits; the kernel then returns early and its outputs are
+ *      undefined).  Read it after synchronising the stream.
+ * A session whose segments are all empty is a caller error: its rows are
+ * written as zero with lse = -inf.
+ * Requirements: head_dim in {64, 128}; 1 <= n_seg <= SR_MAX_SEG; every cap a
+ * positive multiple of SR_TILE; q_cap >= 1.
+ */
+typedef struct {
+    int32_t n_seg;
+    int32_t cap[SR_MAX_SEG];    /* tokens, multiples of SR_TILE */
+} sr_kv_layout;
+
+int sr_chunk_attention_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+                           const sr_kv_layout *layout, const int32_t *kv_len_dev,
+                           const int32_t *q_len_dev, int32_t n_batch, int32_t n_heads,
+                           int32_t head_dim, int32_t q_cap, float softmax_scale,
+                           int32_t *status_dev, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SR_H_ */

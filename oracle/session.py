@@ -34,9 +34,15 @@ def pooled_tier(spec, frames_k, frames_v, ph: int, pw: int):
     return pk.reshape(F * cells, H, D), pv.reshape(F * cells, H, D)
 
 
-def session_kv(spec, inp) -> List[Dict]:
-    """Segments in buffer order: dicts with name, k (pre-RoPE), v [n, H, D] fp64
-    and pos [n, 3] fp64."""
+def session_kv(spec, inp, heads: Optional[Sequence[int]] = None) -> List[Dict]:
+    """Segments in buffer order: dicts with name, k (pre-RoPE), v [n, H', D]
+    fp64 and pos [n, 3] fp64, for the selected heads (default all; heads are
+    independent, so a subset only skips work)."""
+    if heads is not None:
+        sel = list(heads)
+        inp = type(inp)(inp.prompt_k[:, sel], inp.prompt_v[:, sel], [t[:, sel] for t in inp.ctx_k],
+                        [t[:, sel] for t in inp.ctx_v], inp.q[:, sel], inp.k[:, sel], inp.v[:, sel])
+        spec = type(spec)(**{**spec.__dict__, "n_heads": len(sel)})
     H, D = spec.n_heads, spec.head_dim
     segs = {name: {"name": name, "k": [], "v": [], "pos": []} for name in layout.segment_names(spec)}
     segs["prompt"]["k"].append(_f64(inp.prompt_k))
@@ -76,9 +82,9 @@ def session_reference(spec, inp, heads: Optional[Sequence[int]] = None,
     chunk queries ``rows`` (default all) and ``heads`` (default all)."""
     H, D = spec.n_heads, spec.head_dim
     heads = list(range(H)) if heads is None else list(heads)
-    segs = session_kv(spec, inp)
-    k_all = np.concatenate([s["k"][:, heads] for s in segs])
-    v_all = np.concatenate([s["v"][:, heads] for s in segs])
+    segs = session_kv(spec, inp, heads)
+    k_all = np.concatenate([s["k"] for s in segs])
+    v_all = np.concatenate([s["v"] for s in segs])
     p_all = np.concatenate([s["pos"] for s in segs])
     k_rot = rope3d(k_all, p_all, spec.rope_split, spec.rope_base)
     q = _f64(inp.q)[:, heads]

@@ -1,0 +1,202 @@
+// api.cu -- extern "C" entry points of libsr.so: argument validation,
+// tensor-map creation and dispatch to the sm_100a kernels.  Nothing here
+// allocates device memory or synchronises with the device.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "sr_internal.h"
+
+namespace sr {
+
+namespace {
+thread_local char g_last_error[512] = "";
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+std::once_flag g_encode_once;
+EncodeTiledFn g_encode = nullptr;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool stride_ok(int64_t s) { return s % 8 == 0; }
+}  // namespace
+
+int set_error(int code, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int set_cuda_error(const char *what, cudaError_t e) {
+    return set_error(SR_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+int make_tmap_bf16_3d(CUtensorMap *tm, const void *base, uint64_t inner, uint64_t rows, uint64_t outer,
+                      uint32_t box_inner, uint32_t box_rows) {
+    std::call_once(g_encode_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    });
+    if (!g_encode) return set_error(SR_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    const cuuint64_t dims[3] = {inner, rows, outer};
+    const cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
+    const cuuint32_t box[3] = {box_inner, box_rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return set_error(SR_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", int(r));
+    return SR_OK;
+}
+
+}  // namespace sr
+
+using namespace sr;
+
+extern "C" {
+
+int sr_version(void) { return SR_VERSION; }
+
+const char *sr_get_last_error(void) { return g_last_error; }
+
+int sr_rope3d_apply(const void *x, void *y, const float *pos, int32_t n_batch, int32_t n_tokens, int32_t n_heads,
+                    int32_t head_dim, const int32_t *n_valid_dev, sr_rope_cfg cfg, float out_scale,
+                    int64_t x_batch_stride, int64_t x_token_stride, int64_t x_head_stride, int64_t y_batch_stride,
+                    int64_t y_token_stride, int64_t y_head_stride, int64_t pos_batch_stride, void *stream) {
+    g_last_error[0] = 0;
+    if (n_batch < 0 || n_tokens < 0 || n_heads < 1 || n_batch > 65535)
+        return set_error(SR_ERR_INVALID_ARG, "rope3d: bad sizes (batch %d, tokens %d, heads %d)", n_batch,
+                         n_tokens, n_heads);
+    if (head_dim != 64 && head_dim != 128) return set_error(SR_ERR_UNSUPPORTED, "rope3d: head_dim must be 64 or 128");
+    if (cfg.d_t < 0 || cfg.d_h < 0 || cfg.d_w < 0 || cfg.d_t % 8 || cfg.d_h % 8 || cfg.d_w % 8 ||
+        cfg.d_t + cfg.d_h + cfg.d_w != head_dim)
+        return set_error(SR_ERR_INVALID_ARG, "rope3d: sub-blocks %d/%d/%d must be multiples of 8 summing to %d",
+                         cfg.d_t, cfg.d_h, cfg.d_w, head_dim);
+    if (!(cfg.base > 0.f)) return set_error(SR_ERR_INVALID_ARG, "rope3d: base must be positive");
+    if (n_batch == 0 || n_tokens == 0) return SR_OK;
+    if (!x || !y) return set_error(SR_ERR_INVALID_ARG, "rope3d: null tensor");
+    if (!aligned16(x) || !aligned16(y))
+        return set_error(SR_ERR_INVALID_ARG, "rope3d: x and y must be 16-byte aligned");
+    if (!stride_ok(x_batch_stride) || !stride_ok(x_token_stride) || !stride_ok(x_head_stride) ||
+        !stride_ok(y_batch_stride) || !stride_ok(y_token_stride) || !stride_ok(y_head_stride))
+        return set_error(SR_ERR_INVALID_ARG, "rope3d: strides must be multiples of 8 elements");
+    if (pos && (reinterpret_cast<uintptr_t>(pos) & 3u))
+        return set_error(SR_ERR_INVALID_ARG, "rope3d: pos must be 4-byte aligned");
+    RopeLaunch l{x, y, pos, n_valid_dev, n_batch, n_tokens, n_heads, head_dim, cfg, out_scale,
+                 x_batch_stride, x_token_stride, x_head_stride, y_batch_stride, y_token_stride, y_head_stride,
+                 pos_batch_stride, static_cast<cudaStream_t>(stream)};
+    return launch_rope3d(l);
+}
+
+int sr_history_compress(const void *k_in, const void *v_in, void *k_out, void *v_out, int32_t n_batch,
+                        int32_t n_frames, int32_t n_heads, int32_t head_dim, sr_pool_cfg cfg, int64_t in_batch_stride,
+                        int64_t in_frame_stride, int64_t in_token_stride, int64_t in_head_stride,
+                        int64_t out_batch_stride, int64_t out_frame_stride, int64_t out_token_stride,
+                        int64_t out_head_stride, const float *frame_t, float *pos_out, int64_t pos_batch_stride,
+                        int32_t *slot_of_src, void *stream) {
+    g_last_error[0] = 0;
+    if (n_batch < 0 || n_frames < 0 || n_heads < 1)
+        return set_error(SR_ERR_INVALID_ARG, "history_compress: bad sizes");
+    if (head_dim != 64 && head_dim != 128)
+        return set_error(SR_ERR_UNSUPPORTED, "history_compress: head_dim must be 64 or 128");
+    if (cfg.grid_h < 1 || cfg.grid_w < 1 || cfg.pool_h < 1 || cfg.pool_w < 1 || cfg.pool_h > 8 || cfg.pool_w > 8)
+        return set_error(SR_ERR_INVALID_ARG, "history_compress: grid >= 1 and 1 <= pool <= 8 required");
+    if (n_batch == 0 || n_frames == 0) return SR_OK;
+    if ((k_in == nullptr) != (k_out == nullptr) || (v_in == nullptr) != (v_out == nullptr))
+        return set_error(SR_ERR_INVALID_ARG, "history_compress: in/out must be both given or both NULL");
+    for (const void *p : {k_in, v_in, static_cast<const void *>(k_out), static_cast<const void *>(v_out)})
+        if (p && !aligned16(p)) return set_error(SR_ERR_INVALID_ARG, "history_compress: tensors must be 16-byte aligned");
+    for (int64_t s : {in_batch_stride, in_frame_stride, in_token_stride, in_head_stride, out_batch_stride,
+                      out_frame_stride, out_token_stride, out_head_stride})
+        if (!stride_ok(s)) return set_error(SR_ERR_INVALID_ARG, "history_compress: strides must be multiples of 8");
+    if (pos_out && !frame_t) return set_error(SR_ERR_INVALID_ARG, "history_compress: pos_out needs frame_t");
+    PoolLaunch l{k_in, v_in, k_out, v_out, n_batch, n_frames, n_heads, head_dim, cfg,
+                 in_batch_stride, in_frame_stride, in_token_stride, in_head_stride,
+                 out_batch_stride, out_frame_stride, out_token_stride, out_head_stride,
+                 frame_t, pos_out, pos_batch_stride, slot_of_src, static_cast<cudaStream_t>(stream)};
+    return launch_history_compress(l);
+}
+
+int sr_kv_append(void *k_buf, void *v_buf, float *pos_buf, int32_t n_batch, int32_t n_heads, int32_t head_dim,
+                 int32_t buf_tokens, int32_t dst_token, const void *k_src, const void *v_src, const float *pos_src,
+                 int32_t n_tokens, const int32_t *n_valid_dev, int64_t src_batch_stride, int64_t src_token_stride,
+                 int64_t src_head_stride, int64_t pos_src_batch_stride, void *stream) {
+    g_last_error[0] = 0;
+    if (n_batch < 0 || n_heads < 1 || n_tokens < 0 || buf_tokens < 0 || dst_token < 0)
+        return set_error(SR_ERR_INVALID_ARG, "kv_append: bad sizes");
+    if (head_dim != 64 && head_dim != 128) return set_error(SR_ERR_UNSUPPORTED, "kv_append: head_dim must be 64 or 128");
+    if (static_cast<int64_t>(dst_token) + n_tokens > buf_tokens)
+        return set_error(SR_ERR_INVALID_ARG, "kv_append: slots [%d, %d) exceed the buffer (%d tokens)", dst_token,
+                         dst_token + n_tokens, buf_tokens);
+    if (n_batch == 0 || n_tokens == 0) return SR_OK;
+    if ((k_src && !k_buf) || (v_src && !v_buf) || (pos_src && !pos_buf))
+        return set_error(SR_ERR_INVALID_ARG, "kv_append: source given without its buffer");
+    for (const void *p : {static_cast<const void *>(k_buf), static_cast<const void *>(v_buf), k_src, v_src})
+        if (p && !aligned16(p)) return set_error(SR_ERR_INVALID_ARG, "kv_append: tensors must be 16-byte aligned");
+    if (!stride_ok(src_batch_stride) || !stride_ok(src_token_stride) || !stride_ok(src_head_stride))
+        return set_error(SR_ERR_INVALID_ARG, "kv_append: strides must be multiples of 8");
+    AppendLaunch l{k_buf, v_buf, pos_buf, n_batch, n_heads, head_dim, buf_tokens, dst_token, k_src, v_src, pos_src,
+                   n_tokens, n_valid_dev, src_batch_stride, src_token_stride, src_head_stride, pos_src_batch_stride,
+                   static_cast<cudaStream_t>(stream)};
+    return launch_kv_append(l);
+}
+
+int sr_chunk_attention_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+                           const sr_kv_layout *layout, const int32_t *kv_len_dev, const int32_t *q_len_dev,
+                           int32_t n_batch, int32_t n_heads, int32_t head_dim, int32_t q_cap, float softmax_scale,
+                           int32_t *status_dev, void *stream) {
+    g_last_error[0] = 0;
+    if (!layout) return set_error(SR_ERR_INVALID_ARG, "chunk_attention: layout is NULL");
+    if (head_dim != 64 && head_dim != 128)
+        return set_error(SR_ERR_UNSUPPORTED, "chunk_attention: head_dim must be 64 or 128");
+    if (n_batch < 0 || n_batch > 65535 || n_heads < 1 || n_heads > 65535 || q_cap < 1)
+        return set_error(SR_ERR_INVALID_ARG, "chunk_attention: bad sizes (batch %d, heads %d, q_cap %d)", n_batch,
+                         n_heads, q_cap);
+    if (layout->n_seg < 1 || layout->n_seg > SR_MAX_SEG)
+        return set_error(SR_ERR_INVALID_ARG, "chunk_attention: n_seg must be in [1, %d]", SR_MAX_SEG);
+    int64_t kv_tokens = 0;
+    for (int s = 0; s < layout->n_seg; ++s) {
+        if (layout->cap[s] < SR_TILE || layout->cap[s] % SR_TILE)
+            return set_error(SR_ERR_INVALID_ARG, "chunk_attention: cap[%d] = %d is not a positive multiple of %d", s,
+                             layout->cap[s], SR_TILE);
+        kv_tokens += layout->cap[s];
+    }
+    if (kv_tokens > (int64_t(1) << 31) - 1) return set_error(SR_ERR_INVALID_ARG, "chunk_attention: buffer too long");
+    if (!(softmax_scale > 0.f)) return set_error(SR_ERR_INVALID_ARG, "chunk_attention: softmax_scale must be > 0");
+    if (n_batch == 0) return SR_OK;
+    if (!q || !k || !v || !o || !kv_len_dev || !q_len_dev)
+        return set_error(SR_ERR_INVALID_ARG, "chunk_attention: null tensor");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+        return set_error(SR_ERR_INVALID_ARG, "chunk_attention: q, k, v, o must be 16-byte aligned");
+    AttnLaunch a{};
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.o = o;
+    a.lse = lse;
+    a.kv_len = kv_len_dev;
+    a.q_len = q_len_dev;
+    a.status = status_dev;
+    for (int s = 0; s < SR_MAX_SEG; ++s) a.cap[s] = s < layout->n_seg ? layout->cap[s] : 0;
+    a.n_seg = layout->n_seg;
+    a.n_batch = n_batch;
+    a.n_heads = n_heads;
+    a.head_dim = head_dim;
+    a.q_cap = q_cap;
+    a.kv_tokens = kv_tokens;
+    a.softmax_scale = softmax_scale;
+    a.stream = static_cast<cudaStream_t>(stream);
+    return launch_chunk_attention(a);
+}
+
+}  // extern "C"

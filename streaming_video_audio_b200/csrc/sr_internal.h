@@ -1,0 +1,75 @@
+// sr_internal.h -- host-side declarations shared by the libsr.so sources.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/sr.h"
+
+namespace sr {
+
+// Record a thread-local error message and return `code`.
+int set_error(int code, const char *fmt, ...);
+int set_cuda_error(const char *what, cudaError_t e);
+
+// 3-D bf16 tensor map over [outer][rows][inner] (inner contiguous), box
+// {box_inner, box_rows, 1}, 128-byte swizzle, zero fill out of bounds.
+int make_tmap_bf16_3d(CUtensorMap *tm, const void *base, uint64_t inner, uint64_t rows, uint64_t outer,
+                      uint32_t box_inner, uint32_t box_rows);
+
+struct AttnLaunch {
+    const void *q, *k, *v;
+    void *o;
+    float *lse;
+    const int32_t *kv_len, *q_len;
+    int32_t *status;
+    int32_t cap[SR_MAX_SEG];
+    int32_t n_seg, n_batch, n_heads, head_dim, q_cap;
+    int64_t kv_tokens;
+    float softmax_scale;
+    cudaStream_t stream;
+};
+int launch_chunk_attention(const AttnLaunch &a);
+
+struct RopeLaunch {
+    const void *x;
+    void *y;
+    const float *pos;
+    const int32_t *n_valid;
+    int32_t n_batch, n_tokens, n_heads, head_dim;
+    sr_rope_cfg cfg;
+    float out_scale;
+    int64_t xb, xt, xh, yb, yt, yh, pb;
+    cudaStream_t stream;
+};
+int launch_rope3d(const RopeLaunch &a);
+
+struct PoolLaunch {
+    const void *k_in, *v_in;
+    void *k_out, *v_out;
+    int32_t n_batch, n_frames, n_heads, head_dim;
+    sr_pool_cfg cfg;
+    int64_t ib, i_f, it, ih, ob, o_f, ot, oh;
+    const float *frame_t;
+    float *pos_out;
+    int64_t pos_b;
+    int32_t *slot_of_src;
+    cudaStream_t stream;
+};
+int launch_history_compress(const PoolLaunch &a);
+
+struct AppendLaunch {
+    void *k_buf, *v_buf;
+    float *pos_buf;
+    int32_t n_batch, n_heads, head_dim, buf_tokens, dst_token;
+    const void *k_src, *v_src;
+    const float *pos_src;
+    int32_t n_tokens;
+    const int32_t *n_valid;
+    int64_t sb, st, sh, psb;
+    cudaStream_t stream;
+};
+int launch_kv_append(const AppendLaunch &a);
+
+}  // namespace sr

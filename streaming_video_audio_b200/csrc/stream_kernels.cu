@@ -1,0 +1,313 @@
+// stream_kernels.cu -- the HBM-bound steps of the streaming attention layer:
+// 3-D RoPE + re-layout (QK-prep), history-tier pooling and KV append.
+//
+// All three move 16-byte vectors (8 bf16) per thread; a warp covers whole
+// 256-byte head rows (D = 128) so every DRAM sector it touches is used
+// completely.  They do no tensor-core work: their roofline is HBM bandwidth.
+#include <cmath>
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "sr_device.cuh"
+#include "sr_internal.h"
+
+namespace sr {
+
+namespace {
+
+__device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8]) {
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 v = __bfloat1622float2(h[i]);
+        f[2 * i] = v.x;
+        f[2 * i + 1] = v.y;
+    }
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
+    uint4 u;
+    u.x = pack_bf16x2(f[0], f[1]);
+    u.y = pack_bf16x2(f[2], f[3]);
+    u.z = pack_bf16x2(f[4], f[5]);
+    u.w = pack_bf16x2(f[6], f[7]);
+    return u;
+}
+
+// ============================================================== 3-D RoPE
+// Per pair p of the head vector: its axis (0 = t, 1 = h, 2 = w) and
+// theta_p = base^(-2j/d_a) (j = index of the pair inside its axis block),
+// computed on the host in double.
+struct RopeTable {
+    double theta[64];
+    int8_t axis[64];
+};
+
+struct RopeArgs {
+    const __nv_bfloat16 *__restrict__ x;
+    __nv_bfloat16 *__restrict__ y;
+    const float *__restrict__ pos;
+    const int32_t *__restrict__ n_valid;
+    int32_t n_heads;
+    float out_scale;
+    int64_t xb, xt, xh, yb, yt, yh, pb;
+};
+
+// One CTA per (token, batch).  Thread t handles the 16-byte chunk
+// c = t % (D/8) of heads t/(D/8), t/(D/8) + 128/(D/8), ...: the angles of a
+// token depend on (token, pair) only, so each thread evaluates its four
+// (cos, sin) pairs once, in double precision (angle error independent of
+// the position's magnitude), and reuses them across all heads; the rotation
+// itself runs in fp32.
+template <int D>
+__global__ void __launch_bounds__(128) rope3d_kernel(const RopeArgs a, const RopeTable tab) {
+    constexpr int kChunks = D / 8;
+    constexpr int kHeadsPerPass = 128 / kChunks;
+    const int n = blockIdx.x, b = blockIdx.y;
+    if (a.n_valid && n >= a.n_valid[b]) return;
+    const int c = threadIdx.x % kChunks;
+    const int hp = threadIdx.x / kChunks;
+    float cs[4], sn[4];
+    float pt = 0.f, ph = 0.f, pw = 0.f;
+    if (a.pos) {
+        const float *pp = a.pos + b * a.pb + 3 * static_cast<int64_t>(n);
+        pt = pp[0];
+        ph = pp[1];
+        pw = pp[2];
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int pair = c * 4 + k;
+        const int ax = tab.axis[pair];
+        const double pa = ax == 0 ? pt : (ax == 1 ? ph : pw);
+        double s, co;
+        sincos(pa * tab.theta[pair], &s, &co);
+        cs[k] = static_cast<float>(co * a.out_scale);
+        sn[k] = static_cast<float>(s * a.out_scale);
+    }
+    const __nv_bfloat16 *xt = a.x + b * a.xb + n * a.xt + c * 8;
+    __nv_bfloat16 *yt = a.y + b * a.yb + n * a.yt + c * 8;
+#pragma unroll 4
+    for (int h = hp; h < a.n_heads; h += kHeadsPerPass) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4 *>(xt + h * a.xh));
+        float f[8], g[8];
+        unpack8(u, f);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            g[2 * k] = f[2 * k] * cs[k] - f[2 * k + 1] * sn[k];
+            g[2 * k + 1] = f[2 * k] * sn[k] + f[2 * k + 1] * cs[k];
+        }
+        *reinterpret_cast<uint4 *>(yt + h * a.yh) = pack8(g);
+    }
+}
+
+// ============================================================== pooling
+struct PoolArgs {
+    const __nv_bfloat16 *__restrict__ k_in;
+    const __nv_bfloat16 *__restrict__ v_in;
+    __nv_bfloat16 *__restrict__ k_out;
+    __nv_bfloat16 *__restrict__ v_out;
+    int32_t n_frames, n_heads, grid_h, grid_w, pool_h, pool_w, cells_w, cells;
+    int64_t ib, i_f, it, ih, ob, o_f, ot, oh;
+    const float *__restrict__ frame_t;
+    float *__restrict__ pos_out;
+    int64_t pos_b;
+    int64_t total;   // threads doing work
+};
+
+// One thread per (batch, frame, cell, head, 16-byte chunk); chunk fastest so a
+// warp reads whole 256-byte head rows of each member token.
+template <int D>
+__global__ void __launch_bounds__(256) pool_kernel(const PoolArgs a) {
+    constexpr int kChunks = D / 8;
+    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx >= a.total) return;
+    int64_t rest = idx;
+    const int c = static_cast<int>(rest % kChunks);
+    rest /= kChunks;
+    const int h = static_cast<int>(rest % a.n_heads);
+    rest /= a.n_heads;
+    const int j = static_cast<int>(rest % a.cells);
+    rest /= a.cells;
+    const int f = static_cast<int>(rest % a.n_frames);
+    const int b = static_cast<int>(rest / a.n_frames);
+    const int r = j / a.cells_w, cc = j % a.cells_w;
+    const int r0 = r * a.pool_h, r1 = min(r0 + a.pool_h, a.grid_h);
+    const int c0 = cc * a.pool_w, c1 = min(c0 + a.pool_w, a.grid_w);
+    const float count = static_cast<float>((r1 - r0) * (c1 - c0));
+    const int64_t in_off = b * a.ib + f * a.i_f + h * a.ih + c * 8;
+    const int64_t out_off = b * a.ob + f * a.o_f + j * a.ot + h * a.oh + c * 8;
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {
+        const __nv_bfloat16 *src = which ? a.v_in : a.k_in;
+        __nv_bfloat16 *dst = which ? a.v_out : a.k_out;
+        if (!src) continue;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int rr = r0; rr < r1; ++rr) {
+#pragma unroll 4
+            for (int ci = c0; ci < c1; ++ci) {
+                const uint4 u = __ldg(reinterpret_cast<const uint4 *>(
+                    src + in_off + static_cast<int64_t>(rr * a.grid_w + ci) * a.it));
+                float v[8];
+                unpack8(u, v);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[e] += v[e];
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = acc[e] / count;
+        *reinterpret_cast<uint4 *>(dst + out_off) = pack8(acc);
+    }
+    if (a.pos_out && h == 0 && c == 0) {
+        float *pp = a.pos_out + b * a.pos_b + 3 * (static_cast<int64_t>(f) * a.cells + j);
+        pp[0] = a.frame_t[static_cast<int64_t>(b) * a.n_frames + f];
+        pp[1] = 0.5f * static_cast<float>(r0 + r1 - 1);
+        pp[2] = 0.5f * static_cast<float>(c0 + c1 - 1);
+    }
+}
+
+__global__ void slot_map_kernel(int32_t *slot, int n_frames, int grid_h, int grid_w, int pool_h, int pool_w,
+                                int cells_w, int cells) {
+    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t per = static_cast<int64_t>(grid_h) * grid_w;
+    if (idx >= per * n_frames) return;
+    const int f = static_cast<int>(idx / per);
+    const int i = static_cast<int>(idx % per);
+    const int r = i / grid_w, c = i % grid_w;
+    slot[idx] = f * cells + (r / pool_h) * cells_w + c / pool_w;
+}
+
+// ============================================================== KV append
+struct AppendArgs {
+    __nv_bfloat16 *__restrict__ k_buf;
+    __nv_bfloat16 *__restrict__ v_buf;
+    float *__restrict__ pos_buf;
+    const __nv_bfloat16 *__restrict__ k_src;
+    const __nv_bfloat16 *__restrict__ v_src;
+    const float *__restrict__ pos_src;
+    const int32_t *__restrict__ n_valid;
+    int32_t n_heads, n_tokens, buf_tokens, dst_token;
+    int64_t sb, st, sh, psb;
+    int64_t total;
+};
+
+// One thread per (batch, token, head, 16-byte chunk), chunk then head
+// fastest: reads follow the token-major source, writes are whole 256-byte
+// head rows of the head-major buffer.
+template <int D>
+__global__ void __launch_bounds__(256) append_kernel(const AppendArgs a) {
+    constexpr int kChunks = D / 8;
+    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx >= a.total) return;
+    int64_t rest = idx;
+    const int c = static_cast<int>(rest % kChunks);
+    rest /= kChunks;
+    const int h = static_cast<int>(rest % a.n_heads);
+    rest /= a.n_heads;
+    const int n = static_cast<int>(rest % a.n_tokens);
+    const int b = static_cast<int>(rest / a.n_tokens);
+    if (a.n_valid && n >= a.n_valid[b]) return;
+    const int64_t s_off = b * a.sb + n * a.st + h * a.sh + c * 8;
+    const int64_t d_off =
+        ((static_cast<int64_t>(b) * a.n_heads + h) * a.buf_tokens + a.dst_token + n) * D + c * 8;
+    if (a.k_src)
+        *reinterpret_cast<uint4 *>(a.k_buf + d_off) = __ldg(reinterpret_cast<const uint4 *>(a.k_src + s_off));
+    if (a.v_src)
+        *reinterpret_cast<uint4 *>(a.v_buf + d_off) = __ldg(reinterpret_cast<const uint4 *>(a.v_src + s_off));
+    if (a.pos_src && h == 0 && c == 0) {
+        const float *ps = a.pos_src + b * a.psb + 3 * static_cast<int64_t>(n);
+        float *pd = a.pos_buf + (static_cast<int64_t>(b) * a.buf_tokens + a.dst_token + n) * 3;
+        pd[0] = ps[0];
+        pd[1] = ps[1];
+        pd[2] = ps[2];
+    }
+}
+
+template <int D>
+int rope_launch(const RopeLaunch &l) {
+    RopeTable tab{};
+    const int widths[3] = {l.cfg.d_t, l.cfg.d_h, l.cfg.d_w};
+    int pair = 0;
+    for (int ax = 0; ax < 3; ++ax)
+        for (int j = 0; j < widths[ax] / 2; ++j, ++pair) {
+            tab.axis[pair] = static_cast<int8_t>(ax);
+            tab.theta[pair] = std::pow(static_cast<double>(l.cfg.base), -2.0 * static_cast<double>(j) / widths[ax]);
+        }
+    RopeArgs a{static_cast<const __nv_bfloat16 *>(l.x), static_cast<__nv_bfloat16 *>(l.y), l.pos, l.n_valid,
+               l.n_heads, l.out_scale, l.xb, l.xt, l.xh, l.yb, l.yt, l.yh, l.pb};
+    dim3 grid(l.n_tokens, l.n_batch);
+    rope3d_kernel<D><<<grid, 128, 0, l.stream>>>(a, tab);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SR_OK : set_cuda_error("rope3d launch", e);
+}
+
+template <int D>
+int pool_launch(const PoolLaunch &l) {
+    PoolArgs a{};
+    a.k_in = static_cast<const __nv_bfloat16 *>(l.k_in);
+    a.v_in = static_cast<const __nv_bfloat16 *>(l.v_in);
+    a.k_out = static_cast<__nv_bfloat16 *>(l.k_out);
+    a.v_out = static_cast<__nv_bfloat16 *>(l.v_out);
+    a.n_frames = l.n_frames;
+    a.n_heads = l.n_heads;
+    a.grid_h = l.cfg.grid_h;
+    a.grid_w = l.cfg.grid_w;
+    a.pool_h = l.cfg.pool_h;
+    a.pool_w = l.cfg.pool_w;
+    a.cells_w = (l.cfg.grid_w + l.cfg.pool_w - 1) / l.cfg.pool_w;
+    a.cells = a.cells_w * ((l.cfg.grid_h + l.cfg.pool_h - 1) / l.cfg.pool_h);
+    a.ib = l.ib; a.i_f = l.i_f; a.it = l.it; a.ih = l.ih;
+    a.ob = l.ob; a.o_f = l.o_f; a.ot = l.ot; a.oh = l.oh;
+    a.frame_t = l.frame_t;
+    a.pos_out = l.pos_out;
+    a.pos_b = l.pos_b;
+    a.total = static_cast<int64_t>(l.n_batch) * l.n_frames * a.cells * l.n_heads * (D / 8);
+    if (a.total > 0) {
+        const int64_t blocks = (a.total + 255) / 256;
+        pool_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, l.stream>>>(a);
+    }
+    if (l.slot_of_src) {
+        const int64_t n = static_cast<int64_t>(l.n_frames) * l.cfg.grid_h * l.cfg.grid_w;
+        if (n > 0)
+            slot_map_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, l.stream>>>(
+                l.slot_of_src, l.n_frames, l.cfg.grid_h, l.cfg.grid_w, l.cfg.pool_h, l.cfg.pool_w, a.cells_w,
+                a.cells);
+    }
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SR_OK : set_cuda_error("history_compress launch", e);
+}
+
+template <int D>
+int append_launch(const AppendLaunch &l) {
+    AppendArgs a{};
+    a.k_buf = static_cast<__nv_bfloat16 *>(l.k_buf);
+    a.v_buf = static_cast<__nv_bfloat16 *>(l.v_buf);
+    a.pos_buf = l.pos_buf;
+    a.k_src = static_cast<const __nv_bfloat16 *>(l.k_src);
+    a.v_src = static_cast<const __nv_bfloat16 *>(l.v_src);
+    a.pos_src = l.pos_src;
+    a.n_valid = l.n_valid;
+    a.n_heads = l.n_heads;
+    a.n_tokens = l.n_tokens;
+    a.buf_tokens = l.buf_tokens;
+    a.dst_token = l.dst_token;
+    a.sb = l.sb; a.st = l.st; a.sh = l.sh; a.psb = l.psb;
+    a.total = static_cast<int64_t>(l.n_batch) * l.n_tokens * l.n_heads * (D / 8);
+    const int64_t blocks = (a.total + 255) / 256;
+    append_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, l.stream>>>(a);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SR_OK : set_cuda_error("kv_append launch", e);
+}
+
+}  // namespace
+
+int launch_rope3d(const RopeLaunch &l) { return l.head_dim == 128 ? rope_launch<128>(l) : rope_launch<64>(l); }
+int launch_history_compress(const PoolLaunch &l) {
+    return l.head_dim == 128 ? pool_launch<128>(l) : pool_launch<64>(l);
+}
+int launch_kv_append(const AppendLaunch &l) {
+    return l.head_dim == 128 ? append_launch<128>(l) : append_launch<64>(l);
+}
+
+}  // namespace sr

@@ -1,0 +1,325 @@
+"""Streaming window: persistent per-layer KV buffers, their segment layout and
+the window position template, plus the four-call streaming step.
+
+Sources:
+  * "StreamRender-H3" (molayo1419.me), streaming context section: a sink
+    (initial scene, kept all session) plus recent history; bidirectional
+    attention in the window; the position template of the first window is
+    reused afterwards; inference acceleration section: persistent per-layer KV
+    buffers in the attention kernel's layout, only the dynamic region updated
+    in place, lengths and offsets reused without host-device syncs.
+  * "AlayaRenderer-Flash" (aitrends.kr), key contributions and technical
+    details: three history tiers (recent full resolution, older pooled), the
+    first generated frame kept as the appearance anchor, persistent
+    style-prompt KV in every self-attention.
+  * "MiniMax-H3 deep dive" (fiv.co.kr): audio latents at 40 Hz, 6 latent
+    frames per second, a single token sequence for video and audio.
+
+Readings (the pages leave them open): window-relative positions with the
+chunk's frames at t = 0, 1, ... and the context frames at t = -n .. -1 (the
+sink earliest); audio token i at t = i * 6 / 40, h = w = 0; pooled cells at
+(t, mean member row, mean member col); the prompt unrotated; K is kept
+pre-RoPE in the window (``k_raw``) and rotated into ``k_att`` with the current
+template, so re-positioning never compounds rounding.
+
+Buffer layout (per session, head-major, the attention kernel's layout):
+    [prompt | sink | tier (oldest first) ... | recent | chunk]
+each segment padded to a multiple of 128 tokens; frames are frame-major then
+row-major inside a segment; in the chunk, audio follows video.
+
+A session spec is any object with the attributes of ``workloads.SessionSpec``
+(n_heads, head_dim, rope_split, rope_base, grid_h, grid_w, prompt_len,
+context_video_tokens, sink_frames, tiers, chunk_video_tokens,
+chunk_audio_tokens, latent_fps, audio_rate).
+"""
+from __future__ import annotations
+
+import math
+from typing import List, Optional, Sequence
+
+import numpy as np
+import torch
+
+from . import capi
+
+TILE = capi.SR_TILE
+
+
+def _ceil_div(a: int, b: int) -> int:
+    return -(-a // b)
+
+
+def _frame_sizes(total: int, per: int) -> List[int]:
+    full, rem = divmod(total, per)
+    return [per] * full + ([rem] if rem else [])
+
+
+class SessionPlan:
+    """Per-session structure of the window (host side, no device work)."""
+
+    def __init__(self, spec):
+        self.spec = spec
+        self.H, self.D = int(spec.n_heads), int(spec.head_dim)
+        self.gh, self.gw = int(spec.grid_h), int(spec.grid_w)
+        self.frame_tokens = self.gh * self.gw
+        ctx = _frame_sizes(int(spec.context_video_tokens), self.frame_tokens)
+        n = len(ctx)
+        roles = []
+        i = 0
+        for _ in range(min(int(spec.sink_frames), n)):
+            roles.append(("sink", 1, 1))
+            i += 1
+        for ti, (nf, ph, pw) in enumerate(spec.tiers):
+            for _ in range(nf):
+                if i >= n:
+                    raise ValueError("more tier frames than context frames")
+                roles.append((f"tier{ti}", int(ph), int(pw)))
+                i += 1
+        roles += [("recent", 1, 1)] * (n - i)
+        # (segment, t, pool_h, pool_w, source tokens)
+        self.context = [(roles[f][0], float(f - n), roles[f][1], roles[f][2], ctx[f]) for f in range(n)]
+        self.segments = ["prompt"]
+        if any(r == "sink" for r, *_ in self.context):
+            self.segments.append("sink")
+        self.segments += [f"tier{t}" for t in range(len(spec.tiers))]
+        if any(r == "recent" for r, *_ in self.context):
+            self.segments.append("recent")
+        self.segments.append("chunk")
+        self.lengths = {s: 0 for s in self.segments}
+        self.lengths["prompt"] = int(spec.prompt_len)
+        for role, _, ph, pw, ntok in self.context:
+            if role.startswith("tier"):
+                if ntok != self.frame_tokens:
+                    raise ValueError("pooled frames must be complete")
+                self.lengths[role] += self.cells(ph, pw)
+            else:
+                self.lengths[role] += ntok
+        self.chunk_len = int(spec.chunk_video_tokens) + int(spec.chunk_audio_tokens)
+        self.lengths["chunk"] = self.chunk_len
+
+    def cells(self, ph: int, pw: int) -> int:
+        return _ceil_div(self.gh, ph) * _ceil_div(self.gw, pw)
+
+    def grid_positions(self, t: float, n: int) -> np.ndarray:
+        """(t, row, col) of the first n tokens of a full-resolution frame."""
+        r, c = np.divmod(np.arange(n), self.gw)
+        return np.stack([np.full(n, t), r, c], axis=1).astype(np.float32)
+
+    def chunk_positions(self) -> np.ndarray:
+        sp = self.spec
+        parts = [self.grid_positions(float(f), n)
+                 for f, n in enumerate(_frame_sizes(int(sp.chunk_video_tokens), self.frame_tokens))]
+        na = int(sp.chunk_audio_tokens)
+        ta = np.arange(na, dtype=np.float64) * (float(sp.latent_fps) / float(sp.audio_rate))
+        parts.append(np.stack([ta, np.zeros(na), np.zeros(na)], axis=1).astype(np.float32))
+        return np.concatenate(parts).reshape(-1, 3)
+
+
+class StreamingWindow:
+    """Device state of a batch of streaming sessions for one DiT layer.
+
+    All sessions share the segment names and capacities (the largest valid
+    length per segment, rounded up to 128); their valid lengths may differ
+    (ragged batch).  Buffers are allocated once, zero-filled, and updated in
+    place afterwards.
+    """
+
+    def __init__(self, specs: Sequence, device="cuda"):
+        self.plans = [SessionPlan(s) for s in specs]
+        p0 = self.plans[0]
+        self.B, self.H, self.D = len(self.plans), p0.H, p0.D
+        self.split = tuple(int(x) for x in p0.spec.rope_split)
+        self.base = float(p0.spec.rope_base)
+        for p in self.plans:
+            if (p.H, p.D, p.segments, tuple(p.spec.rope_split)) != (self.H, self.D, p0.segments, self.split):
+                raise ValueError("sessions of one window must share heads, head_dim, RoPE split and segments")
+        self.segments = p0.segments
+        self.caps = [max(TILE, _ceil_div(max(p.lengths[s] for p in self.plans), TILE) * TILE)
+                     for s in self.segments]
+        self.offsets = [int(x) for x in np.cumsum([0] + self.caps[:-1])]
+        self.cap_total = int(sum(self.caps))
+        self.seg = {s: (int(o), int(c)) for s, o, c in zip(self.segments, self.offsets, self.caps)}
+        self.q_cap = max(p.chunk_len for p in self.plans)
+        self.device = torch.device(device)
+        B, H, D, C = self.B, self.H, self.D, self.cap_total
+        kw = dict(device=self.device)
+        self.k_raw = torch.zeros(B, H, C, D, dtype=torch.bfloat16, **kw)
+        self.k_att = torch.zeros(B, H, C, D, dtype=torch.bfloat16, **kw)
+        self.v = torch.zeros(B, H, C, D, dtype=torch.bfloat16, **kw)
+        self.pos = torch.zeros(B, C, 3, dtype=torch.float32, **kw)
+        self.q_att = torch.zeros(B, H, self.q_cap, D, dtype=torch.bfloat16, **kw)
+        self.o = torch.zeros(B, self.q_cap, H, D, dtype=torch.bfloat16, **kw)
+        self.lse = torch.zeros(B, H, self.q_cap, dtype=torch.float32, **kw)
+        self.status = torch.zeros(1, dtype=torch.int32, **kw)
+        lens = np.array([[p.lengths[s] for s in self.segments] for p in self.plans], dtype=np.int32)
+        self.lengths = lens
+        self.kv_len = torch.from_numpy(lens).to(self.device)
+        self.seg_valid = torch.from_numpy(np.ascontiguousarray(lens.T)).to(self.device)   # [n_seg, B]
+        self.q_len = torch.tensor([p.chunk_len for p in self.plans], dtype=torch.int32, device=self.device)
+        qpos = np.zeros((B, self.q_cap, 3), dtype=np.float32)
+        for b, p in enumerate(self.plans):
+            qpos[b, :p.chunk_len] = p.chunk_positions()
+        self.q_pos = torch.from_numpy(qpos).to(self.device)
+        self.scale = 1.0 / math.sqrt(D)
+
+    # ---------------------------------------------------------------- views
+    def seg_view(self, buf: torch.Tensor, name: str) -> torch.Tensor:
+        """[B, cap, H, D] token-major view of one segment of a head-major buffer."""
+        off, cap = self.seg[name]
+        return buf[:, :, off:off + cap].permute(0, 2, 1, 3)
+
+    def valid_mask(self, b: int) -> np.ndarray:
+        m = np.zeros(self.cap_total, dtype=bool)
+        for s, (off, _) in self.seg.items():
+            m[off:off + self.plans[b].lengths[s]] = True
+        return m
+
+    # ---------------------------------------------------------------- window fill
+    def load_window(self, inputs: Sequence, stream=None) -> None:
+        """Fill prompt and context segments of every session from its drawn
+        inputs (``workloads.SessionInputs``-like: prompt_k/v [Lp, H, D], ctx_k/v
+        lists of [tokens, H, D] full-resolution frames, oldest first).  Tier
+        frames are pooled on the device by sr_history_compress."""
+        dev = self.device
+        for b, (plan, inp) in enumerate(zip(self.plans, inputs)):
+            kb, vb, pb = self.k_raw[b:b + 1], self.v[b:b + 1], self.pos[b:b + 1]
+            lp = plan.lengths["prompt"]
+            if lp:
+                capi.sr_kv_append(kb, vb, pb, self.seg["prompt"][0], inp.prompt_k.to(dev)[None],
+                                  inp.prompt_v.to(dev)[None], torch.zeros(1, lp, 3, device=dev), stream=stream)
+            fill = {s: 0 for s in self.segments}
+            f = 0
+            ctx = plan.context
+            while f < len(ctx):
+                role, t, ph, pw, ntok = ctx[f]
+                if role.startswith("tier"):
+                    g = f
+                    while g < len(ctx) and ctx[g][0] == role:
+                        g += 1
+                    nf = g - f
+                    cells = plan.cells(ph, pw)
+                    src_k = torch.stack([inp.ctx_k[i] for i in range(f, g)]).to(dev)[None]
+                    src_v = torch.stack([inp.ctx_v[i] for i in range(f, g)]).to(dev)[None]
+                    off = self.seg[role][0] + fill[role]
+                    n_out = nf * cells
+                    out_k = self.k_raw[b:b + 1, :, off:off + n_out].permute(0, 2, 1, 3).reshape(1, nf, cells, self.H, self.D)
+                    out_v = self.v[b:b + 1, :, off:off + n_out].permute(0, 2, 1, 3).reshape(1, nf, cells, self.H, self.D)
+                    frame_t = torch.tensor([[ctx[i][1] for i in range(f, g)]], dtype=torch.float32, device=dev)
+                    capi.sr_history_compress(src_k, src_v, out_k, out_v, (plan.gh, plan.gw), (ph, pw),
+                                             frame_t=frame_t, pos_out=self.pos[b:b + 1, off:off + n_out],
+                                             stream=stream)
+                    fill[role] += n_out
+                    f = g
+                else:
+                    off = self.seg[role][0] + fill[role]
+                    pos = torch.from_numpy(plan.grid_positions(t, ntok)).to(dev)[None]
+                    capi.sr_kv_append(kb, vb, pb, off, inp.ctx_k[f].to(dev)[None], inp.ctx_v[f].to(dev)[None],
+                                      pos, stream=stream)
+                    fill[role] += ntok
+                    f += 1
+        # the prompt is never re-positioned: rotate (identity) once
+        pv = self.seg_view(self.k_raw, "prompt")
+        capi.sr_rope3d_apply(pv, self.seg_view(self.k_att, "prompt"), None, self.split, self.base,
+                             n_valid=self.seg_valid[0], stream=stream)
+        # chunk positions are the fixed template
+        off = self.seg["chunk"][0]
+        self.pos[:, off:off + self.q_cap].copy_(self.q_pos)
+
+    # ---------------------------------------------------------------- the step
+    def append_chunk(self, k: torch.Tensor, v: torch.Tensor, stream=None) -> None:
+        """a2: chunk K (pre-RoPE) and V [B, q_cap, H, D] into the chunk segment."""
+        capi.sr_kv_append(self.k_raw, self.v, None, self.seg["chunk"][0], k, v, None, n_valid=self.q_len,
+                          stream=stream)
+
+    def rotate(self, q: torch.Tensor, stream=None) -> None:
+        """a3: RoPE of the chunk queries into q_att and of every non-prompt
+        window segment from k_raw into k_att, with the current template."""
+        capi.sr_rope3d_apply(q, self.q_att.permute(0, 2, 1, 3), self.q_pos, self.split, self.base,
+                             n_valid=self.q_len, stream=stream)
+        for si, name in enumerate(self.segments):
+            if name == "prompt":
+                continue
+            off, cap = self.seg[name]
+            capi.sr_rope3d_apply(self.seg_view(self.k_raw, name), self.seg_view(self.k_att, name),
+                                 self.pos[:, off:off + cap], self.split, self.base,
+                                 n_valid=self.seg_valid[si], stream=stream)
+
+    def attend(self, stream=None) -> torch.Tensor:
+        """a4: fused chunk attention -> o [B, q_cap, H, D] (and lse)."""
+        capi.sr_chunk_attention_fwd(self.q_att, self.k_att, self.v, self.o, self.lse, self.caps, self.kv_len,
+                                    self.q_len, self.scale, self.status, stream=stream)
+        return self.o
+
+    def step(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream=None) -> torch.Tensor:
+        """One streaming attention step: a2 -> a3 -> a4 (device tensors
+        [B, q_cap, H, D], token-major, pre-RoPE)."""
+        self.append_chunk(k, v, stream)
+        self.rotate(q, stream)
+        return self.attend(stream)
+
+    def step_from_host(self, q_host: torch.Tensor, k_host: torch.Tensor, v_host: torch.Tensor,
+                       o_host: torch.Tensor, staging=None, stream=None) -> torch.Tensor:
+        """The streaming step for callers holding host tensors: copy the chunk's
+        q, k, v [B, q_cap, H, D] (pinned host memory for asynchronous copies)
+        to the device, run the step, copy o back into ``o_host``.  ``staging``
+        is an optional (q, k, v) triple of device tensors reused across calls.
+        Asynchronous on the current stream; synchronise before reading o_host."""
+        if staging is None:
+            staging = tuple(torch.empty_like(t, device=self.device) for t in (q_host, k_host, v_host))
+        for dst, src in zip(staging, (q_host, k_host, v_host)):
+            dst.copy_(src, non_blocking=True)
+        o = self.step(*staging, stream=stream)
+        o_host.copy_(o, non_blocking=True)
+        return o_host
+
+    def check_status(self) -> None:
+        """Raise if a bounded wait inside the attention kernel gave up
+        (synchronises with the device)."""
+        s = int(self.status.item())
+        if s != 0:
+            self.status.zero_()
+            raise capi.SrError("sr_chunk_attention_fwd", s, "a pipeline wait timed out on the device")
+
+    # ---------------------------------------------------------------- tier aging
+    def tier_boundaries(self):
+        """(source segment, destination tier, source grid, pool) for every tier
+        boundary, destination-oldest first: each tier is fed by the next
+        newer tier, the newest tier by the recent frames."""
+        plan = self.plans[0]
+        tiers = [f"tier{i}" for i in range(len(plan.spec.tiers))]
+        if not tiers or "recent" not in self.segments:
+            return []
+        grid = {"recent": (plan.gh, plan.gw)}
+        for i, (_, ph, pw) in enumerate(plan.spec.tiers):
+            grid[tiers[i]] = (_ceil_div(plan.gh, ph), _ceil_div(plan.gw, pw))
+        out = []
+        for i, dst in enumerate(tiers):
+            src = tiers[i + 1] if i + 1 < len(tiers) else "recent"
+            (gh, gw), (dh, dw) = grid[src], grid[dst]
+            out.append((src, dst, (gh, gw), (_ceil_div(gh, dh), _ceil_div(gw, dw))))
+        return out
+
+    def age_tiers(self, step_index: int, n_frames: int, stream=None) -> None:
+        """a1 in steady-state streaming: at every tier boundary the n_frames
+        oldest frames of the newer segment are pooled into the older tier
+        (oldest boundary first, so a tier's frames are consumed before they
+        are overwritten).  Frames live in ring slots that advance with
+        step_index; segment lengths stay constant (full rings).  K and V are
+        pooled pre-RoPE; positions are rewritten by the next re-positioning."""
+        for src, dst, (gh, gw), (ph, pw) in self.tier_boundaries():
+            src_tok = gh * gw
+            dst_tok = _ceil_div(gh, ph) * _ceil_div(gw, pw)
+            n_src = self.plans[0].lengths[src] // src_tok
+            n_dst = self.plans[0].lengths[dst] // dst_tok
+            fs = (step_index * n_frames) % n_src
+            fd = (step_index * n_frames) % n_dst
+            nf = min(n_frames, n_src - fs, n_dst - fd)
+            so = self.seg[src][0] + fs * src_tok
+            do = self.seg[dst][0] + fd * dst_tok
+
+            def frames(buf, off, tok):
+                return buf[:, :, off:off + nf * tok].permute(0, 2, 1, 3).reshape(self.B, nf, tok, self.H, self.D)
+
+            capi.sr_history_compress(frames(self.k_raw, so, src_tok), frames(self.v, so, src_tok),
+                                     frames(self.k_raw, do, dst_tok), frames(self.v, do, dst_tok),
+                                     (gh, gw), (ph, pw), stream=stream)

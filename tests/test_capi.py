@@ -1,0 +1,80 @@
+"""CPU checks of the C-ABI boundary: the library loads without a GPU, exports
+every function include/sr.h declares, and rejects bad arguments on the host
+before launching anything (no compute calls are made here)."""
+import ctypes
+
+import pytest
+
+from streaming_video_audio_b200 import capi
+
+EXPECTED = {"sr_version", "sr_get_last_error", "sr_rope3d_apply", "sr_history_compress", "sr_kv_append",
+            "sr_chunk_attention_fwd"}
+
+
+def test_header_declares_the_boundary():
+    assert EXPECTED <= set(capi.declared_functions())
+
+
+def test_library_exports_every_declared_symbol():
+    lib = capi.load()
+    for name in capi.declared_functions():
+        assert hasattr(lib, name), name
+    assert capi.sr_version() == 1
+
+
+def _err(lib):
+    return lib.sr_get_last_error().decode()
+
+
+def test_attention_rejects_bad_arguments_on_host():
+    lib = capi.load()
+    lay = capi.make_layout([128, 256])
+    args = lambda **kw: dict(dict(q=None, k=None, v=None, o=None, lse=None, lay=ctypes.byref(lay), kl=None, ql=None,
+                                  B=1, H=1, D=128, qcap=100, scale=0.1), **kw)
+
+    def call(a):
+        return lib.sr_chunk_attention_fwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["lay"], a["kl"], a["ql"],
+                                          a["B"], a["H"], a["D"], a["qcap"], a["scale"], None, None)
+
+    assert call(args(D=96)) == capi.SR_ERR_UNSUPPORTED and "head_dim" in _err(lib)
+    assert call(args(qcap=0)) == capi.SR_ERR_INVALID_ARG
+    assert call(args(scale=0.0)) == capi.SR_ERR_INVALID_ARG
+    assert call(args()) == capi.SR_ERR_INVALID_ARG and "null" in _err(lib)
+    bad = capi.make_layout([100])
+    assert call(args(lay=ctypes.byref(bad))) == capi.SR_ERR_INVALID_ARG and "multiple" in _err(lib)
+    assert call(args(B=0)) == capi.SR_OK                       # zero work: nothing launched
+    assert call(args(q=16, k=32, v=48, o=72, kl=1, ql=1)) == capi.SR_ERR_INVALID_ARG   # misaligned o
+    assert "aligned" in _err(lib)
+
+
+def test_rope_rejects_bad_arguments_on_host():
+    lib = capi.load()
+    cfg = capi.sr_rope_cfg(10000.0, 32, 48, 48)
+    call = lambda D=128, c=cfg, x=16, y=32, xs=(0, 5120, 128): lib.sr_rope3d_apply(
+        x, y, None, 1, 4, 40, D, None, c, 1.0, xs[0], xs[1], xs[2], 0, 5120, 128, 0, None)
+    assert call(D=64) == capi.SR_ERR_INVALID_ARG                          # split does not sum to D
+    assert call(c=capi.sr_rope_cfg(10000.0, 30, 50, 48)) == capi.SR_ERR_INVALID_ARG
+    assert call(x=8) == capi.SR_ERR_INVALID_ARG                           # misaligned
+    assert call(xs=(0, 5120, 100)) == capi.SR_ERR_INVALID_ARG             # stride not a multiple of 8
+    assert lib.sr_rope3d_apply(16, 32, None, 1, 0, 40, 128, None, cfg, 1.0, 0, 0, 0, 0, 0, 0, 0, None) == capi.SR_OK
+
+
+def test_append_and_pool_reject_bad_arguments_on_host():
+    lib = capi.load()
+    rc = lib.sr_kv_append(16, 32, None, 1, 2, 128, 256, 200, 48, 64, None, 100, None, 0, 256, 128, 0, None)
+    assert rc == capi.SR_ERR_INVALID_ARG and "exceed" in _err(lib)
+    cfg = capi.sr_pool_cfg(24, 42, 9, 2)
+    rc = lib.sr_history_compress(16, 32, 48, 64, 1, 1, 2, 128, cfg, 0, 0, 256, 128, 0, 0, 256, 128,
+                                 None, None, 0, None, None)
+    assert rc == capi.SR_ERR_INVALID_ARG
+    cfg = capi.sr_pool_cfg(24, 42, 2, 2)
+    rc = lib.sr_history_compress(16, None, 48, 64, 1, 1, 2, 128, cfg, 0, 0, 256, 128, 0, 0, 256, 128,
+                                 None, None, 0, None, None)
+    assert rc == capi.SR_ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(capi, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(capi, "_lib", None)
+    with pytest.raises(RuntimeError, match="libsr.so not found"):
+        capi.load()

@@ -1,0 +1,229 @@
+"""Kernel-level parity of the CUDA path against the fp64 oracle (needs a B200).
+
+Inputs come from ``workloads`` (seeded draws); expected values only from
+``oracle``.  Every call goes through the C ABI (``capi``)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from streaming_video_audio_b200 import capi
+from tests.helpers import ATTN_MAX_ABS, ATTN_MEAN_ABS, LSE_ABS, attn_errors, ulp_diff_bf16
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+# ---------------------------------------------------------------- RoPE (a3)
+def assert_rope_close(got, ref, x):
+    """Within one bf16 ulp of the fp64 rotation, except where the rotated
+    component nearly cancels: there the fp32 rotation's own error (a few
+    2^-24 of the pair's norm) may exceed half an ulp of the tiny result, so
+    an absolute 2^-21 * |pair| is allowed."""
+    ulps = ulp_diff_bf16(got, ref)
+    xd = x.double().numpy()
+    pair = np.repeat(np.hypot(xd[..., 0::2], xd[..., 1::2]), 2, axis=-1)
+    err = np.abs(got.double().numpy() - ref)
+    assert np.all((ulps <= 1) | (err <= 2.0 ** -21 * pair))
+
+
+
+@pytest.mark.parametrize("D,split,H,N", [(128, (32, 48, 48), 40, 300), (64, (16, 24, 24), 3, 77),
+                                         (128, (32, 48, 48), 5, 1)])
+def test_rope_token_major_to_head_major(D, split, H, N):
+    B = 2
+    x = workloads.draw_tensor((B, N, H, D), seed=1)
+    pos = torch.stack([workloads.draw_positions(N, seed=2 + b) for b in range(B)])
+    pos[:, :, 0] = torch.round(pos[:, :, 0] * 20) / 20          # mixes integer and fractional t
+    y = torch.full((B, H, N + 5, D), 7.0, dtype=torch.bfloat16, device=DEV)
+    n_valid = torch.tensor([N, max(1, N - 3)], dtype=torch.int32, device=DEV)
+    capi.sr_rope3d_apply(x.to(DEV), y[:, :, :N].permute(0, 2, 1, 3), pos.to(DEV), split, n_valid=n_valid)
+    torch.cuda.synchronize()
+    for b in range(B):
+        nv = int(n_valid[b])
+        ref = oracle.rope3d(x[b, :nv], pos[b, :nv].double(), split)        # [nv, H, D]
+        got = y[b, :, :nv].permute(1, 0, 2).cpu()
+        assert_rope_close(got, ref, x[b, :nv])
+        # skipped tokens and padding slots untouched
+        assert torch.all(y[b, :, nv:].float().cpu() == 7.0)
+
+
+def test_rope_zero_position_copy_and_scale():
+    D, split, H, N = 128, (32, 48, 48), 4, 130
+    x = workloads.draw_tensor((1, N, H, D), seed=3)
+    y = torch.empty(1, N, H, D, dtype=torch.bfloat16, device=DEV)
+    capi.sr_rope3d_apply(x.to(DEV), y, None, split)
+    assert torch.equal(y.cpu(), x)
+    capi.sr_rope3d_apply(x.to(DEV), y, None, split, out_scale=0.5)
+    assert torch.equal(y.cpu(), (x.float() * 0.5).to(torch.bfloat16))
+
+
+# ---------------------------------------------------------------- pooling (a1)
+@pytest.mark.parametrize("grid,pool,D", [((24, 42), (2, 2), 128), ((24, 42), (4, 4), 128), ((12, 21), (2, 2), 128),
+                                         ((5, 7), (4, 4), 64), ((6, 8), (3, 2), 64)])
+def test_history_compress(grid, pool, D):
+    gh, gw = grid
+    ph, pw = pool
+    B, F, H = 2, 3, 3
+    cells = (-(-gh // ph)) * (-(-gw // pw))
+    k = workloads.draw_tensor((B, F, gh * gw, H, D), seed=4)
+    v = workloads.draw_tensor((B, F, gh * gw, H, D), seed=5)
+    ko = torch.zeros(B, F, cells, H, D, dtype=torch.bfloat16, device=DEV)
+    vo = torch.zeros_like(ko)
+    frame_t = torch.tensor([[-9.0, -8.0, -7.0], [-3.0, -2.0, -1.0]], device=DEV)
+    pos = torch.zeros(B, F * cells, 3, device=DEV)
+    slot = torch.full((F * gh * gw,), -1, dtype=torch.int32, device=DEV)
+    capi.sr_history_compress(k.to(DEV), v.to(DEV), ko, vo, grid, pool, frame_t=frame_t, pos_out=pos,
+                             slot_of_src=slot)
+    torch.cuda.synchronize()
+    for b in range(B):
+        for src, out in ((k, ko), (v, vo)):
+            ref = oracle.pool(src[b].reshape(F, gh, gw, H, D), ph, pw).reshape(F, cells, H, D)
+            assert ulp_diff_bf16(out[b].cpu(), ref).max() <= 1
+    # positions and the slot map are index arithmetic: bit-exact
+    from oracle import layout
+    cell_pos = np.array([(mr, mc) for (_, _, _, _, mr, mc) in layout.pooled_cells(gh, gw, ph, pw)])
+    exp = np.zeros((B, F * cells, 3), np.float32)
+    for b in range(B):
+        for f in range(F):
+            exp[b, f * cells:(f + 1) * cells, 0] = frame_t[b, f].item()
+            exp[b, f * cells:(f + 1) * cells, 1:] = cell_pos
+    assert np.array_equal(pos.cpu().numpy(), exp)
+    exp_slot = np.empty(F * gh * gw, np.int32)
+    for f in range(F):
+        for j, (r0, r1, c0, c1, _, _) in enumerate(layout.pooled_cells(gh, gw, ph, pw)):
+            for r in range(r0, r1):
+                for c in range(c0, c1):
+                    exp_slot[f * gh * gw + r * gw + c] = f * cells + j
+    assert np.array_equal(slot.cpu().numpy(), exp_slot)
+
+
+def test_history_compress_two_stage_matches_direct():
+    """T2 -> T3 re-pooling on the device vs direct 4x4 pooling of the
+    full-resolution frames (equal in exact arithmetic on a 24x42 grid).  The
+    bound follows from the two roundings: each T2 value is off by at most
+    2^-9 of its magnitude, their mean by at most 2^-9 max|T2|, and the final
+    rounding adds 2^-9 |T3|."""
+    H, D = 4, 128
+    k = workloads.draw_tensor((1, 2, 1008, H, D), seed=6)
+    t2 = torch.zeros(1, 2, 252, H, D, dtype=torch.bfloat16, device=DEV)
+    t3 = torch.zeros(1, 2, 66, H, D, dtype=torch.bfloat16, device=DEV)
+    capi.sr_history_compress(k.to(DEV), None, t2, None, (24, 42), (2, 2))
+    capi.sr_history_compress(t2, None, t3, None, (12, 21), (2, 2))
+    ref = oracle.pool(k[0].reshape(2, 24, 42, H, D), 4, 4).reshape(2, 66, H, D)
+    t2max = np.abs(oracle.pool(k[0].reshape(2, 24, 42, H, D), 2, 2)).max()
+    err = np.abs(t3[0].cpu().double().numpy() - ref)
+    assert np.all(err <= 2.0 ** -9 * (t2max + np.abs(ref)) + 1e-12)
+
+
+# ---------------------------------------------------------------- append (a2)
+def test_kv_append_exact_and_in_place():
+    B, H, D, cap, N = 2, 5, 128, 512, 200
+    kb = torch.zeros(B, H, cap, D, dtype=torch.bfloat16, device=DEV)
+    vb = torch.zeros_like(kb)
+    pb = torch.zeros(B, cap, 3, device=DEV)
+    ks = workloads.draw_tensor((B, N, H, D), seed=7)
+    vs = workloads.draw_tensor((B, N, H, D), seed=8)
+    ps = torch.stack([workloads.draw_positions(N, seed=9), workloads.draw_positions(N, seed=10)])
+    nv = torch.tensor([N, 150], dtype=torch.int32, device=DEV)
+    capi.sr_kv_append(kb, vb, pb, 100, ks.to(DEV), vs.to(DEV), ps.to(DEV), n_valid=nv)
+    torch.cuda.synchronize()
+    for b, n in enumerate((N, 150)):
+        assert torch.equal(kb[b, :, 100:100 + n].cpu(), ks[b, :n].permute(1, 0, 2))
+        assert torch.equal(vb[b, :, 100:100 + n].cpu(), vs[b, :n].permute(1, 0, 2))
+        assert torch.equal(pb[b, 100:100 + n].cpu(), ps[b, :n])
+        assert not kb[b, :, :100].any() and not kb[b, :, 100 + n:].any()
+        assert not pb[b, 100 + n:].any()
+
+
+# ---------------------------------------------------------------- attention (a4)
+def _draw_case(D, H, caps, lens, q_len, seed, perturb_padding=False):
+    """Seeded bf16 q/k/v in the kernel's layout (padding optionally filled with
+    large finite garbage)."""
+    B = len(lens)
+    C = sum(caps)
+    q_cap = max(q_len)
+    q = workloads.draw_tensor((B, H, q_cap, D), seed=seed)
+    k = workloads.draw_tensor((B, H, C, D), seed=seed + 1, scale=0.7)
+    v = workloads.draw_tensor((B, H, C, D), seed=seed + 2)
+    if perturb_padding:
+        rng = np.random.default_rng(seed + 3)
+        for b in range(B):
+            off = 0
+            for cap, n in zip(caps, lens[b]):
+                pad = slice(off + n, off + cap)
+                for t in (k, v):
+                    shape = t[b, :, pad].shape
+                    t[b, :, pad] = torch.from_numpy(rng.uniform(-60, 60, shape).astype(np.float32)).to(torch.bfloat16)
+                off += cap
+    return q, k, v
+
+
+def _run_attention(q, k, v, caps, lens, q_len):
+    B, H, q_cap, D = q.shape
+    o = torch.full((B, q_cap, H, D), 3.0, dtype=torch.bfloat16, device=DEV)
+    lse = torch.zeros(B, H, q_cap, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    capi.sr_chunk_attention_fwd(q.to(DEV).contiguous(), k.to(DEV).contiguous(), v.to(DEV).contiguous(), o, lse,
+                                caps, torch.tensor(lens, dtype=torch.int32, device=DEV),
+                                torch.tensor(q_len, dtype=torch.int32, device=DEV), 1 / math.sqrt(D), status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    return o.cpu(), lse.cpu()
+
+
+def _attention_case(D, H, caps, lens, q_len, seed, perturb_padding=False):
+    q, k, v = _draw_case(D, H, caps, lens, q_len, seed, perturb_padding)
+    o, lse = _run_attention(q, k, v, caps, lens, q_len)
+    return q, k, v, o, lse
+
+
+def _valid_kv(k, v, b, h, caps, lens_b):
+    idx, off = [], 0
+    for cap, n in zip(caps, lens_b):
+        idx += list(range(off, off + n))
+        off += cap
+    return k[b, h, idx], v[b, h, idx]
+
+
+@pytest.mark.parametrize("D,H,caps,lens,q_len", [
+    (128, 2, [256, 512, 384], [[200, 300, 333]], [333]),
+    (64, 1, [128, 128, 128], [[16, 96, 100]], [100]),
+    (128, 3, [128, 1024, 256], [[1, 1000, 129], [128, 7, 256], [0, 513, 255]], [129, 256, 255]),
+    (64, 2, [256, 256], [[256, 256], [1, 0]], [200, 1]),
+])
+def test_attention_matches_oracle(D, H, caps, lens, q_len):
+    q, k, v, o, lse = _attention_case(D, H, caps, lens, q_len, seed=20)
+    for b in range(len(lens)):
+        for h in range(H):
+            kk, vv = _valid_kv(k, v, b, h, caps, lens[b])
+            ro, rl = oracle.attention(q[b, h, :q_len[b]], kk, vv, 1 / math.sqrt(D))
+            mx, mean = attn_errors(o[b, :q_len[b], h], ro)
+            assert mx <= ATTN_MAX_ABS and mean <= ATTN_MEAN_ABS, (b, h, mx, mean)
+            assert np.abs(lse[b, h, :q_len[b]].double().numpy() - rl).max() <= LSE_ABS
+        # rows beyond q_len untouched
+        assert torch.all(o[b, q_len[b]:] == 3.0)
+
+
+def test_attention_ignores_padding_and_other_sessions():
+    """Finite garbage in padded slots and the presence of other sessions in
+    the batch change no output bit."""
+    D, H, caps = 128, 2, [128, 384, 256]
+    lens = [[100, 300, 200], [128, 257, 129]]
+    args = (D, H, caps, lens, [200, 129])
+    _, _, _, o1, l1 = _attention_case(*args, seed=30)
+    _, _, _, o2, l2 = _attention_case(*args, seed=30, perturb_padding=True)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    q, k, v = _draw_case(*args, seed=30)
+    o3, l3 = _run_attention(q[:1], k[:1], v[:1], caps, lens[:1], [200])
+    assert torch.equal(o3[0, :200], o1[0, :200]) and torch.equal(l3[0, :, :200], l1[0, :, :200])
+
+
+def test_attention_all_segments_empty_writes_zeros():
+    D, H, caps = 64, 1, [128, 128]
+    _, _, _, o, lse = _attention_case(D, H, caps, [[0, 0]], [5], seed=40)
+    assert torch.all(o[0, :5] == 0) and torch.all(torch.isinf(lse[0, 0, :5]))
