@@ -12,23 +12,27 @@
 // "AlayaRenderer-Flash" (aitrends.kr) -- methodology (past chunks as clean
 // tokens; persistent style-prompt KV in every self-attention layer).
 //
-// Design (one CTA = one 128-row query tile of one (session, head)):
-//   warp 0      TMA producer: Q once, then K and V tiles (128 tokens) into a
-//               2-stage ring each, walking the segments' valid tiles only.
-//   warp 1      TMEM owner + single-thread tcgen05.mma issuer:
-//                 S_j = Q K_j^T   (M=128, N=128, K=D; S double-buffered in TMEM)
-//                 O  += P_j V_j   (M=128, N=D, K=128; O resident in TMEM)
-//               S_{j+1} is issued before waiting for P_j so QK^T overlaps
-//               the softmax of the previous tile.
-//   warps 2..5  softmax: one thread per query row reads its S row from TMEM,
-//               masks the segment tail, keeps an fp32 running max/sum in the
-//               log2 domain, writes P (bf16) into a 128B-swizzled shared
-//               tile and rescales O in TMEM only when the row max grew by
-//               more than 2^8 (lazy rescale; exact because the final
-//               normalisation uses the same stale max).  Epilogue: O / l ->
-//               bf16 token-major output, LSE.
-// Every wait is bounded (sr_device.cuh): a stuck pipeline sets the status word
-// and the CTA returns instead of hanging.
+// Design (one CTA = two 128-row query tiles Q0, Q1 of one (session, head),
+// sharing every K/V tile; 16 warps):
+//   warps 0-3   softmax of Q0, warps 4-7 softmax of Q1 (one thread per query
+//               row): read the S row from TMEM, mask the segment tail, keep an
+//               fp32 running max/sum in the log2 domain, write P (bf16 pairs)
+//               back into TMEM over the S columns.  The max only moves when it
+//               grows by more than 2^8 (lazy rescale: exact, the final
+//               normalisation uses the same stale max).
+//   warps 8-11  correction: rescale O_t in TMEM when a row's max moved, and the
+//               epilogue (O / l -> bf16 token-major, LSE).
+//   warp 12     TMA producer: Q0, Q1 once, then K and V tiles (128 tokens) into
+//               two-stage rings, walking only the segments' valid tiles.
+//   warp 13     TMEM owner + single-thread tcgen05.mma issuer, ping-pong order
+//                 PV0(j), S0(j+1) = Q0 K(j+1)^T, PV1(j), S1(j+1)
+//               so the tensor core works on one tile while the other tile's
+//               softmax runs.  S = Q K^T reads both operands from shared memory;
+//               O += P V reads P from TMEM (A operand) and V from shared memory.
+// TMEM: S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512) (fp32 columns); P_t
+// aliases the first 64 columns of S_t.  Every wait is bounded
+// (sr_device.cuh): a stuck pipeline sets the status word and the CTA returns
+// instead of hanging.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -42,12 +46,19 @@ namespace {
 
 constexpr int kTileM = 128;
 constexpr int kTileN = 128;
+constexpr int kQTiles = 2;               // query tiles per CTA
 constexpr int kStages = 2;
-constexpr int kThreads = 192;
+constexpr int kThreads = 512;
+constexpr int kWarpTma = 12, kWarpMma = 13;
 constexpr int kPanelBytes = 128 * 128;   // 128 rows x 128 bytes (64 bf16), one swizzle-128B panel
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO = 256;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
+// Registers per thread after reallocation (launch: 65536 / 512 = 128 each):
+// 2 x 128 x 160 + 128 x 88 + 128 x 104 = 65536 (the launch total; no spills).
+constexpr int kRegSoftmax = 160, kRegCorrection = 88, kRegOther = 104;
+
+__host__ __device__ constexpr uint32_t tmem_s(int t) { return static_cast<uint32_t>(t) * 128u; }
+__host__ __device__ constexpr uint32_t tmem_o(int t) { return 256u + static_cast<uint32_t>(t) * 128u; }
 
 struct AttnParams {
     __nv_bfloat16 *o;
@@ -68,13 +79,14 @@ struct Smem {
     static constexpr int kPanels = D / 64;
     static constexpr int kTileBytes = kPanels * kPanelBytes;
     static constexpr int kQ = 0;
-    static constexpr int kK = kQ + kTileBytes;
+    static constexpr int kK = kQ + kQTiles * kTileBytes;
     static constexpr int kV = kK + kStages * kTileBytes;
-    static constexpr int kP = kV + kStages * kTileBytes;
-    static constexpr int kBar = kP + 2 * kPanelBytes;
-    static constexpr int kNumBars = 1 + 4 * kStages + 2 + 1 + 1;
+    static constexpr int kBar = kV + kStages * kTileBytes;
+    // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], alpha_ready[2], p_full[2], o_done[2]
+    static constexpr int kNumBars = 1 + 4 * kStages + 4 * kQTiles;
     static constexpr int kMisc = kBar + kNumBars * 8;
-    static constexpr int kEnd = kMisc + 16 + 12 * SR_MAX_SEG;
+    static constexpr int kRow = kMisc + 16 + 12 * SR_MAX_SEG;   // float alpha[2][128], l[2][128], m[2][128]
+    static constexpr int kEnd = kRow + 3 * kQTiles * kTileM * 4;
     static constexpr int kAlloc = kEnd + 1024;   // slack for manual 1024-byte alignment
 };
 
@@ -95,6 +107,11 @@ struct TileWalk {
     }
 };
 
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                          int32_t *status) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, status));
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -103,9 +120,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
-    const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int q_len = p.q_len[b];
-    const int q0 = qt * kTileM;
+    const int q0 = qb * kQTiles * kTileM;
     if (q0 >= q_len) return;   // uniform for the whole CTA
     const int bh = b * p.n_heads + h;
 
@@ -115,15 +132,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *k_empty = k_full + kStages;
     uint64_t *v_full = k_empty + kStages;
     uint64_t *v_empty = v_full + kStages;
-    uint64_t *s_full = v_empty + kStages;   // [2]
-    uint64_t *p_full = s_full + 2;
-    uint64_t *o_done = p_full + 1;
+    uint64_t *s_full = v_empty + kStages;        // [2] MMA -> softmax t
+    uint64_t *alpha_ready = s_full + kQTiles;    // [2] softmax t -> correction
+    uint64_t *p_full = alpha_ready + kQTiles;    // [2] softmax t + correction -> MMA
+    uint64_t *o_done = p_full + kQTiles;         // [2] MMA (PV_t) -> correction
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
     int *n_tiles_s = reinterpret_cast<int *>(smem + L::kMisc + 8);
     int *seg_ntile = reinterpret_cast<int *>(smem + L::kMisc + 16);
     int *seg_len = seg_ntile + SR_MAX_SEG;
     int *seg_start = seg_len + SR_MAX_SEG;
+    float *row_alpha = reinterpret_cast<float *>(smem + L::kRow);   // [2][128]
+    float *row_l = row_alpha + kQTiles * kTileM;                     // [2][128]
+    float *row_m = row_l + kQTiles * kTileM;                         // [2][128]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -135,10 +156,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&v_full[i], 1);
             mbar_init(&v_empty[i], 1);
         }
-        mbar_init(&s_full[0], 1);
-        mbar_init(&s_full[1], 1);
-        mbar_init(p_full, 4);   // one arrival per softmax warp
-        mbar_init(o_done, 1);
+        for (int t = 0; t < kQTiles; ++t) {
+            mbar_init(&s_full[t], 1);
+            mbar_init(&alpha_ready[t], 4);   // the four softmax warps of tile t
+            mbar_init(&p_full[t], 8);        // four softmax + four correction warps
+            mbar_init(&o_done[t], 1);
+        }
         *abort_flag = 0;
         int total = 0;
 #pragma unroll
@@ -153,7 +176,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         *n_tiles_s = total;
         fence_mbarrier_init();
     }
-    if (warp == 1) {
+    if (warp == kWarpMma) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
@@ -163,109 +186,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tmem_slot;
     const int n_tiles = *n_tiles_s;
     const int n_seg = p.n_seg;
+    const float sl2 = p.scale_log2;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
-        if (lane == 0 && n_tiles > 0) {
-            tma_prefetch_desc(&tmQ);
-            tma_prefetch_desc(&tmK);
-            tma_prefetch_desc(&tmV);
-            mbar_expect_tx(q_full, L::kTileBytes);
-#pragma unroll
-            for (int pn = 0; pn < L::kPanels; ++pn)
-                tma_load_3d(smem + L::kQ + pn * kPanelBytes, &tmQ, pn * 64, q0, bh, q_full);
-            TileWalk w;
-            w.first(seg_ntile, n_seg);
-            for (int j = 0; j < n_tiles; ++j, w.next(seg_ntile, n_seg)) {
-                const int st = j % kStages;
-                const uint32_t ph = (j / kStages) & 1;
-                const int row0 = seg_start[w.s] + w.t * kTileN;
-                if (!mbar_wait(&k_empty[st], ph ^ 1, abort_flag, p.status)) break;
-                mbar_expect_tx(&k_full[st], L::kTileBytes);
-#pragma unroll
-                for (int pn = 0; pn < L::kPanels; ++pn)
-                    tma_load_3d(smem + L::kK + st * L::kTileBytes + pn * kPanelBytes, &tmK, pn * 64, row0, bh,
-                                &k_full[st]);
-                if (!mbar_wait(&v_empty[st], ph ^ 1, abort_flag, p.status)) break;
-                mbar_expect_tx(&v_full[st], L::kTileBytes);
-#pragma unroll
-                for (int pn = 0; pn < L::kPanels; ++pn)
-                    tma_load_3d(smem + L::kV + st * L::kTileBytes + pn * kPanelBytes, &tmV, pn * 64, row0, bh,
-                                &v_full[st]);
-            }
-        }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0 && n_tiles > 0) {
-            constexpr uint32_t idesc_qk = umma_idesc_bf16(kTileM, kTileN, false, false);
-            constexpr uint32_t idesc_pv = umma_idesc_bf16(kTileM, D, false, true);
-            const uint32_t q_base = smem_u32(smem + L::kQ);
-            const uint32_t k_base = smem_u32(smem + L::kK);
-            const uint32_t v_base = smem_u32(smem + L::kV);
-            const uint32_t p_base = smem_u32(smem + L::kP);
-            auto issue_qk = [&](int j) {
-                const int st = j % kStages;
-                const uint32_t s_col = (j & 1) ? kTmemS1 : kTmemS0;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kPanelBytes + (kk & 3) * 32;
-                    const uint64_t a = umma_desc_sw128(q_base + off, 16, 1024);
-                    const uint64_t bdesc = umma_desc_sw128(k_base + st * L::kTileBytes + off, 16, 1024);
-                    umma_bf16_ss(tmem + s_col, a, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
-                }
-                umma_commit(&k_empty[st]);
-                umma_commit(&s_full[j & 1]);
-            };
-            bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
-            if (ok) ok = mbar_wait(&k_full[0], 0, abort_flag, p.status);
-            if (ok) {
-                tc_fence_after();
-                issue_qk(0);
-            }
-            for (int j = 0; ok && j < n_tiles; ++j) {
-                if (j + 1 < n_tiles) {
-                    if (!(ok = mbar_wait(&k_full[(j + 1) % kStages], ((j + 1) / kStages) & 1, abort_flag,
-                                         p.status)))
-                        break;
-                    tc_fence_after();
-                    issue_qk(j + 1);
-                }
-                if (!(ok = mbar_wait(p_full, j & 1, abort_flag, p.status))) break;
-                const int st = j % kStages;
-                if (!(ok = mbar_wait(&v_full[st], (j / kStages) & 1, abort_flag, p.status))) break;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < kTileN / 16; ++kk) {
-                    const uint64_t a =
-                        umma_desc_sw128(p_base + (kk >> 2) * kPanelBytes + (kk & 3) * 32, 16, 1024);
-                    const uint64_t bdesc =
-                        umma_desc_sw128(v_base + st * L::kTileBytes + kk * 2048, kPanelBytes, 1024);
-                    umma_bf16_ss(tmem + kTmemO, a, bdesc, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-                }
-                umma_commit(&v_empty[st]);
-                umma_commit(o_done);
-            }
-        }
-    } else {
-        // ------------------------------------------------------------ softmax + epilogue
-        const int quarter = warp & 3;   // TMEM lanes this warp may access
+    if (warp < 4 * kQTiles) {
+        // ================================================================ softmax of tile t
+        regs_increase<kRegSoftmax>();
+        const int t = warp >> 2;
+        const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-        const uint32_t p_base = smem_u32(smem + L::kP);
-        const float sl2 = p.scale_log2;
+        const uint32_t s_addr = tmem + lane_base + tmem_s(t);
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
         TileWalk w;
         w.first(seg_ntile, n_seg);
         for (int j = 0; j < n_tiles; ++j, w.next(seg_ntile, n_seg)) {
             const int valid = min(kTileN, seg_len[w.s] - w.t * kTileN);
-            ok = __all_sync(0xffffffffu, mbar_wait(&s_full[j & 1], (j >> 1) & 1, abort_flag, p.status));
-            if (!ok) break;   // warp-uniform: the TMEM loads below are warp-collective
+            if (!(ok = warp_wait(&s_full[t], j & 1, abort_flag, p.status))) break;
             tc_fence_after();
             float s[kTileN];
             {
                 uint32_t r[4][32];
-                const uint32_t s_addr = tmem + lane_base + ((j & 1) ? kTmemS1 : kTmemS0);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, r[c]);
                 tmem_wait_ld();
@@ -274,69 +215,112 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(r[c][e]);
             }
-            float mx = -INFINITY;
+            if (valid < kTileN) {
 #pragma unroll
-            for (int c = 0; c < kTileN; ++c) mx = fmaxf(mx, c < valid ? s[c] : -INFINITY);
+                for (int c = 0; c < kTileN; ++c) s[c] = c < valid ? s[c] : -INFINITY;
+            }
+            // row max: eight independent chains, then a tree
+            float mx8[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mx8[i] = s[i];
+#pragma unroll
+            for (int c = 8; c < kTileN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
             const float m_new = fmaxf(m_run, mx * sl2);
             const bool need = m_new > m_run + kRescaleThreshold;
             const float m_use = need ? m_new : m_run;
             const float alpha = need ? fast_exp2(m_run - m_use) : 1.0f;
-            float sum = 0.f;
+            float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int c = 0; c < kTileN; ++c) {
-                const float pc = c < valid ? fast_exp2(fmaf(s[c], sl2, -m_use)) : 0.f;
-                s[c] = pc;
-                sum += pc;
+                s[c] = fast_exp2(fmaf(s[c], sl2, -m_use));
+                sum8[c & 7] += s[c];
             }
+            const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
             l_run = l_run * alpha + sum;
             m_run = m_use;
-            if (j > 0) {
-                ok = __all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, abort_flag, p.status));
-                if (!ok) break;
-                tc_fence_after();
-            }
-            // P row -> swizzled shared tile: panel c/64, 16-byte chunk index XOR (row % 8)
+            row_alpha[t * kTileM + row] = alpha;
+            // P (bf16 pairs) over the first 64 columns of S_t
 #pragma unroll
-            for (int ch = 0; ch < kTileN / 8; ++ch) {
-                const uint32_t addr =
-                    p_base + (ch >> 3) * kPanelBytes + row * 128 + ((((ch & 7) ^ (row & 7))) << 4);
-                st_shared_v4(addr, pack_bf16x2(s[8 * ch + 0], s[8 * ch + 1]), pack_bf16x2(s[8 * ch + 2], s[8 * ch + 3]),
-                             pack_bf16x2(s[8 * ch + 4], s[8 * ch + 5]), pack_bf16x2(s[8 * ch + 6], s[8 * ch + 7]));
-            }
-            if (j > 0 && __any_sync(0xffffffffu, need)) {
+            for (int half = 0; half < 2; ++half) {
+                uint32_t pk[32];
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t r[32];
-                    const uint32_t o_addr = tmem + lane_base + kTmemO + c * 32;
-                    tmem_ld32(o_addr, r);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-                    tmem_st32(o_addr, r);
-                }
-                tmem_wait_st();
+                for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(s[half * 64 + 2 * e], s[half * 64 + 2 * e + 1]);
+                tmem_st32(s_addr + half * 32, pk);
             }
-            fence_proxy_async_smem();
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_full);
+            if (lane == 0) {
+                mbar_arrive(&alpha_ready[t]);
+                mbar_arrive(&p_full[t]);
+            }
+        }
+        // hand the row statistics to the epilogue (one more alpha_ready phase)
+        row_l[t * kTileM + row] = l_run;
+        row_m[t * kTileM + row] = m_run;
+        __syncwarp();
+        if (ok && lane == 0) mbar_arrive(&alpha_ready[t]);
+    } else if (warp < 4 * kQTiles + 4) {
+        // ================================================================ correction + epilogue
+        regs_decrease<kRegCorrection>();
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+        bool ok = true;
+        for (int j = 0; ok && j < n_tiles; ++j) {
+#pragma unroll
+            for (int t = 0; t < kQTiles; ++t) {
+                if (!(ok = warp_wait(&alpha_ready[t], j & 1, abort_flag, p.status))) break;
+                const float alpha = row_alpha[t * kTileM + row];
+                if (j > 0) {
+                    // PV_t(j-1) must have landed before O_t is touched; waiting on
+                    // every phase also keeps the parity waits from lagging.
+                    if (!(ok = warp_wait(&o_done[t], (j - 1) & 1, abort_flag, p.status))) break;
+                    if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+                        tc_fence_after();
+#pragma unroll
+                        for (int c = 0; c < D / 32; ++c) {
+                            uint32_t r[32];
+                            const uint32_t o_addr = tmem + lane_base + tmem_o(t) + c * 32;
+                            tmem_ld32(o_addr, r);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+                            tmem_st32(o_addr, r);
+                        }
+                        tmem_wait_st();
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_full[t]);
+            }
         }
         // ---------------------------------------------------------------- epilogue
-        const int grow = q0 + row;
-        const bool row_ok = grow < q_len;
-        __nv_bfloat16 *orow = p.o + ((static_cast<size_t>(b) * p.q_cap + grow) * p.n_heads + h) * D;
-        if (n_tiles == 0) {
-            if (row_ok) {
-                for (int d = 0; d < D; d += 8) *reinterpret_cast<uint4 *>(orow + d) = make_uint4(0, 0, 0, 0);
-                if (p.lse) p.lse[static_cast<size_t>(bh) * p.q_cap + grow] = -INFINITY;
+#pragma unroll
+        for (int t = 0; t < kQTiles; ++t) {
+            const int grow = q0 + t * kTileM + row;
+            const bool row_ok = grow < q_len;
+            __nv_bfloat16 *orow = p.o + ((static_cast<size_t>(b) * p.q_cap + grow) * p.n_heads + h) * D;
+            if (n_tiles == 0) {
+                if (row_ok) {
+                    for (int d = 0; d < D; d += 8) *reinterpret_cast<uint4 *>(orow + d) = make_uint4(0, 0, 0, 0);
+                    if (p.lse) p.lse[static_cast<size_t>(bh) * p.q_cap + grow] = -INFINITY;
+                }
+                continue;
             }
-        } else if (ok && __all_sync(0xffffffffu, mbar_wait(o_done, (n_tiles - 1) & 1, abort_flag, p.status))) {
+            if (!ok) break;
+            if (!(ok = warp_wait(&alpha_ready[t], n_tiles & 1, abort_flag, p.status))) break;
+            if (!(ok = warp_wait(&o_done[t], (n_tiles - 1) & 1, abort_flag, p.status))) break;
             tc_fence_after();
-            const float inv_l = 1.0f / l_run;
+            const float l_row = row_l[t * kTileM + row];
+            const float inv_l = 1.0f / l_row;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t r[32];
-                tmem_ld32(tmem + lane_base + kTmemO + c * 32, r);
+                tmem_ld32(tmem + lane_base + tmem_o(t) + c * 32, r);
                 tmem_wait_ld();
                 if (row_ok) {
 #pragma unroll
@@ -351,13 +335,107 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             if (row_ok && p.lse)
-                p.lse[static_cast<size_t>(bh) * p.q_cap + grow] = (m_run + log2f(l_run)) * 0.69314718055994531f;
+                p.lse[static_cast<size_t>(bh) * p.q_cap + grow] =
+                    (row_m[t * kTileM + row] + log2f(l_row)) * 0.69314718055994531f;
+        }
+    } else {
+        regs_decrease<kRegOther>();
+        if (warp == kWarpTma) {
+            // ============================================================ TMA producer
+            if (lane == 0 && n_tiles > 0) {
+                tma_prefetch_desc(&tmQ);
+                tma_prefetch_desc(&tmK);
+                tma_prefetch_desc(&tmV);
+                mbar_expect_tx(q_full, kQTiles * L::kTileBytes);
+#pragma unroll
+                for (int t = 0; t < kQTiles; ++t)
+#pragma unroll
+                    for (int pn = 0; pn < L::kPanels; ++pn)
+                        tma_load_3d(smem + L::kQ + t * L::kTileBytes + pn * kPanelBytes, &tmQ, pn * 64,
+                                    q0 + t * kTileM, bh, q_full);
+                TileWalk w;
+                w.first(seg_ntile, n_seg);
+                for (int j = 0; j < n_tiles; ++j, w.next(seg_ntile, n_seg)) {
+                    const int st = j % kStages;
+                    const uint32_t ph = (j / kStages) & 1;
+                    const int row0 = seg_start[w.s] + w.t * kTileN;
+                    if (!mbar_wait(&k_empty[st], ph ^ 1, abort_flag, p.status)) break;
+                    mbar_expect_tx(&k_full[st], L::kTileBytes);
+#pragma unroll
+                    for (int pn = 0; pn < L::kPanels; ++pn)
+                        tma_load_3d(smem + L::kK + st * L::kTileBytes + pn * kPanelBytes, &tmK, pn * 64, row0, bh,
+                                    &k_full[st]);
+                    if (!mbar_wait(&v_empty[st], ph ^ 1, abort_flag, p.status)) break;
+                    mbar_expect_tx(&v_full[st], L::kTileBytes);
+#pragma unroll
+                    for (int pn = 0; pn < L::kPanels; ++pn)
+                        tma_load_3d(smem + L::kV + st * L::kTileBytes + pn * kPanelBytes, &tmV, pn * 64, row0, bh,
+                                    &v_full[st]);
+                }
+            }
+        } else if (warp == kWarpMma) {
+            // ============================================================ MMA issuer
+            if (lane == 0 && n_tiles > 0) {
+                constexpr uint32_t idesc_qk = umma_idesc_bf16(kTileM, kTileN, false, false);
+                constexpr uint32_t idesc_pv = umma_idesc_bf16(kTileM, D, false, true);
+                const uint32_t q_base = smem_u32(smem + L::kQ);
+                const uint32_t k_base = smem_u32(smem + L::kK);
+                const uint32_t v_base = smem_u32(smem + L::kV);
+                auto issue_qk = [&](int t, int st) {
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * kPanelBytes + (kk & 3) * 32;
+                        const uint64_t a = umma_desc_sw128(q_base + t * L::kTileBytes + off, 16, 1024);
+                        const uint64_t bd = umma_desc_sw128(k_base + st * L::kTileBytes + off, 16, 1024);
+                        umma_bf16_ss(tmem + tmem_s(t), a, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(&s_full[t]);
+                };
+                auto issue_pv = [&](int t, int st, bool acc) {
+#pragma unroll
+                    for (int kk = 0; kk < kTileN / 16; ++kk) {
+                        const uint64_t bd = umma_desc_sw128(v_base + st * L::kTileBytes + kk * 2048, kPanelBytes, 1024);
+                        umma_bf16_ts(tmem + tmem_o(t), tmem + tmem_s(t) + kk * 8, bd, idesc_pv,
+                                     (acc || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(&o_done[t]);
+                };
+                bool ok = mbar_wait(q_full, 0, abort_flag, p.status) && mbar_wait(&k_full[0], 0, abort_flag, p.status);
+                if (ok) {
+                    tc_fence_after();
+                    issue_qk(0, 0);
+                    issue_qk(1, 0);
+                    umma_commit(&k_empty[0]);
+                }
+                for (int j = 0; ok && j < n_tiles; ++j) {
+                    const int st = j % kStages;
+                    const int st1 = (j + 1) % kStages;
+                    const bool more = j + 1 < n_tiles;
+                    if (!(ok = mbar_wait(&v_full[st], (j / kStages) & 1, abort_flag, p.status))) break;
+                    if (!(ok = mbar_wait(&p_full[0], j & 1, abort_flag, p.status))) break;
+                    tc_fence_after();
+                    issue_pv(0, st, j > 0);
+                    if (more) {
+                        if (!(ok = mbar_wait(&k_full[st1], ((j + 1) / kStages) & 1, abort_flag, p.status))) break;
+                        tc_fence_after();
+                        issue_qk(0, st1);
+                    }
+                    if (!(ok = mbar_wait(&p_full[1], j & 1, abort_flag, p.status))) break;
+                    tc_fence_after();
+                    issue_pv(1, st, j > 0);
+                    umma_commit(&v_empty[st]);
+                    if (more) {
+                        issue_qk(1, st1);
+                        umma_commit(&k_empty[st1]);
+                    }
+                }
+            }
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kWarpMma) {
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
@@ -398,7 +476,7 @@ int launch(const AttnLaunch &a) {
         if (e != cudaSuccess) return set_cuda_error("cudaFuncSetAttribute(chunk_attention)", e);
         if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
-    dim3 grid((a.q_cap + kTileM - 1) / kTileM, a.n_heads, a.n_batch);
+    dim3 grid((a.q_cap + kQTiles * kTileM - 1) / (kQTiles * kTileM), a.n_heads, a.n_batch);
     chunk_attention_kernel<D><<<grid, kThreads, L::kAlloc, a.stream>>>(tq, tk, tv, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return set_cuda_error("chunk_attention launch", e);
