@@ -187,6 +187,15 @@ int sr_kv_append(void *k_buf, void *v_buf, float *pos_buf,
  * kv_len_dev int32 [n_batch][layout->n_seg] (device), 0 <= len <= cap
  * q_len_dev  int32 [n_batch] (device), 1 <= q_len <= q_cap; rows >= q_len are
  *      neither computed into o nor lse.
+ * workspace  optional caller-owned device scratch of workspace_bytes >=
+ *      sr_chunk_attention_workspace_bytes(n_batch, n_heads, head_dim, q_cap)
+ *      bytes (16-byte aligned), or NULL.  With it, when the (session, head,
+ *      256-row query block) units do not fill whole waves of the GPU's SMs,
+ *      the units of the last partial wave are split along the KV tiles and
+ *      their fp32 partial results are merged by a second kernel on the same
+ *      stream; without it every unit runs whole.  Calls that share one
+ *      workspace must be ordered (same stream).  Results of the two schedules
+ *      agree to fp32 rounding.
  * status_dev optional int32 (device): left untouched on success; set to
  *      SR_ERR_DEVICE_TIMEOUT if a pipeline wait inside the kernel gave up
  *      (bounded waits; the kernel then returns early and its outputs are
@@ -205,7 +214,13 @@ int sr_chunk_attention_fwd(const void *q, const void *k, const void *v, void *o,
                            const sr_kv_layout *layout, const int32_t *kv_len_dev,
                            const int32_t *q_len_dev, int32_t n_batch, int32_t n_heads,
                            int32_t head_dim, int32_t q_cap, float softmax_scale,
+                           void *workspace, size_t workspace_bytes,
                            int32_t *status_dev, void *stream);
+
+/* Bytes of workspace sr_chunk_attention_fwd can use for this problem on the
+ * current device (0 if it would never split, or on invalid sizes).  Host
+ * only; reads the device's SM count (no allocation, no synchronisation). */
+size_t sr_chunk_attention_workspace_bytes(int32_t n_batch, int32_t n_heads, int32_t head_dim, int32_t q_cap);
 
 #ifdef __cplusplus
 }

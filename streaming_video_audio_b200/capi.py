@@ -61,7 +61,8 @@ _SIGS = {
     "sr_kv_append": ([_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _i32, _vp,
                       _i64, _i64, _i64, _i64, _vp], ctypes.c_int),
     "sr_chunk_attention_fwd": ([_vp, _vp, _vp, _vp, _vp, ctypes.POINTER(sr_kv_layout), _vp, _vp, _i32, _i32,
-                                _i32, _i32, _f32, _vp, _vp], ctypes.c_int),
+                                _i32, _i32, _f32, _vp, ctypes.c_size_t, _vp, _vp], ctypes.c_int),
+    "sr_chunk_attention_workspace_bytes": ([_i32, _i32, _i32, _i32], ctypes.c_size_t),
 }
 
 
@@ -234,13 +235,19 @@ def make_layout(caps: Sequence[int]) -> sr_kv_layout:
     return lay
 
 
+def sr_chunk_attention_workspace_bytes(n_batch: int, n_heads: int, head_dim: int, q_cap: int) -> int:
+    return int(load().sr_chunk_attention_workspace_bytes(n_batch, n_heads, head_dim, q_cap))
+
+
 def sr_chunk_attention_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
                            lse: Optional[torch.Tensor], caps: Sequence[int], kv_len: torch.Tensor,
                            q_len: torch.Tensor, softmax_scale: float, status: Optional[torch.Tensor] = None,
-                           stream=None) -> None:
+                           workspace: Optional[torch.Tensor] = None, stream=None) -> None:
     """q [B, H, q_cap, D], k, v [B, H, sum(caps), D], o [B, q_cap, H, D] (bf16,
     contiguous); lse fp32 [B, H, q_cap] or None; kv_len int32 [B, n_seg];
-    q_len int32 [B]; status int32 [>=1] or None."""
+    q_len int32 [B]; status int32 [>=1] or None; workspace: a contiguous
+    device byte tensor of at least sr_chunk_attention_workspace_bytes(...)
+    bytes, or None (no KV split of the last partial wave)."""
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
         _cuda(t, torch.bfloat16, n)
         if not t.is_contiguous():
@@ -261,7 +268,12 @@ def sr_chunk_attention_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o:
         raise ValueError("kv_len must be contiguous int32 [B, n_seg]")
     if tuple(q_len.shape) != (B,) or not q_len.is_contiguous():
         raise ValueError("q_len must be contiguous int32 [B]")
+    ws_bytes = 0
+    if workspace is not None:
+        if not workspace.is_cuda or not workspace.is_contiguous():
+            raise ValueError("workspace must be a contiguous CUDA tensor")
+        ws_bytes = workspace.numel() * workspace.element_size()
     lay = make_layout(caps)
     _check("sr_chunk_attention_fwd", load().sr_chunk_attention_fwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), ctypes.byref(lay), _ptr(kv_len), _ptr(q_len),
-        B, H, D, q_cap, float(softmax_scale), _ptr(status), _stream(stream)))
+        B, H, D, q_cap, float(softmax_scale), _ptr(workspace), ws_bytes, _ptr(status), _stream(stream)))

@@ -151,10 +151,15 @@ int sr_kv_append(void *k_buf, void *v_buf, float *pos_buf, int32_t n_batch, int3
     return launch_kv_append(l);
 }
 
+size_t sr_chunk_attention_workspace_bytes(int32_t n_batch, int32_t n_heads, int32_t head_dim, int32_t q_cap) {
+    if (n_batch < 1 || n_heads < 1 || q_cap < 1 || (head_dim != 64 && head_dim != 128)) return 0;
+    return attention_schedule(n_batch, n_heads, head_dim, q_cap, attention_sm_count()).workspace_bytes;
+}
+
 int sr_chunk_attention_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
                            const sr_kv_layout *layout, const int32_t *kv_len_dev, const int32_t *q_len_dev,
                            int32_t n_batch, int32_t n_heads, int32_t head_dim, int32_t q_cap, float softmax_scale,
-                           int32_t *status_dev, void *stream) {
+                           void *workspace, size_t workspace_bytes, int32_t *status_dev, void *stream) {
     g_last_error[0] = 0;
     if (!layout) return set_error(SR_ERR_INVALID_ARG, "chunk_attention: layout is NULL");
     if (head_dim != 64 && head_dim != 128)
@@ -195,6 +200,10 @@ int sr_chunk_attention_fwd(const void *q, const void *k, const void *v, void *o,
     a.q_cap = q_cap;
     a.kv_tokens = kv_tokens;
     a.softmax_scale = softmax_scale;
+    if (workspace && !aligned16(workspace))
+        return set_error(SR_ERR_INVALID_ARG, "chunk_attention: workspace must be 16-byte aligned");
+    a.workspace = workspace;
+    a.workspace_bytes = workspace ? workspace_bytes : 0;
     a.stream = static_cast<cudaStream_t>(stream);
     return launch_chunk_attention(a);
 }

@@ -72,6 +72,14 @@ struct AttnParams {
     int32_t n_heads;
     int32_t q_cap;
     float scale_log2;        // softmax_scale * log2(e)
+    // work list: items [0, n_full) are whole units (one per CTA); the
+    // remaining units are each split into `split` KV ranges whose partial
+    // results meet in the workspace
+    int32_t qb_per_head;     // 256-row query blocks per (session, head)
+    int32_t n_full;
+    int32_t split;
+    float *ws_o;             // [slot][2][128][D] unnormalised partial O (log2-domain max m, sum l)
+    float *ws_ml;            // [slot][m | l][2][128]
 };
 
 template <int D>
@@ -82,10 +90,11 @@ struct Smem {
     static constexpr int kK = kQ + kQTiles * kTileBytes;
     static constexpr int kV = kK + kStages * kTileBytes;
     static constexpr int kBar = kV + kStages * kTileBytes;
-    // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], alpha_ready[2], p_full[2], o_done[2]
-    static constexpr int kNumBars = 1 + 4 * kStages + 4 * kQTiles;
+    // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S],
+    // s_full[2], alpha_ready[2], p_full[2], o_done[2], stats_ready[2]
+    static constexpr int kNumBars = 1 + 4 * kStages + 5 * kQTiles;
     static constexpr int kMisc = kBar + kNumBars * 8;
-    static constexpr int kRow = kMisc + 16 + 12 * SR_MAX_SEG;   // float alpha[2][128], l[2][128], m[2][128]
+    static constexpr int kRow = kMisc + 16 + 12 * SR_MAX_SEG + 16;   // float alpha[2][128], l[2][128], m[2][128]
     static constexpr int kEnd = kRow + 3 * kQTiles * kTileM * 4;
     static constexpr int kAlloc = kEnd + 1024;   // slack for manual 1024-byte alignment
 };
@@ -107,6 +116,8 @@ struct TileWalk {
     }
 };
 
+
+
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                           int32_t *status) {
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, status));
@@ -120,11 +131,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
-    const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    // ---- work item -> (unit, KV part)
+    const int item = blockIdx.x;
+    int unit, part = 0, split = 1;
+    if (item < p.n_full) {
+        unit = item;
+    } else {
+        split = p.split;
+        unit = p.n_full + (item - p.n_full) / split;
+        part = (item - p.n_full) % split;
+    }
+    const int qb = unit % p.qb_per_head;
+    const int bh = unit / p.qb_per_head;
+    const int h = bh % p.n_heads, b = bh / p.n_heads;
     const int q_len = p.q_len[b];
     const int q0 = qb * kQTiles * kTileM;
     if (q0 >= q_len) return;   // uniform for the whole CTA
-    const int bh = b * p.n_heads + h;
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBar);
     uint64_t *q_full = bars;
@@ -136,12 +158,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *alpha_ready = s_full + kQTiles;    // [2] softmax t -> correction
     uint64_t *p_full = alpha_ready + kQTiles;    // [2] softmax t + correction -> MMA
     uint64_t *o_done = p_full + kQTiles;         // [2] MMA (PV_t) -> correction
+    // [2] softmax t -> epilogue: final row max / sum.  A barrier of its own:
+    // a second arrival on alpha_ready could complete two phases before the
+    // correction warps wait on the first, and parity waits would alias.
+    uint64_t *stats_ready = o_done + kQTiles;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
     int *n_tiles_s = reinterpret_cast<int *>(smem + L::kMisc + 8);
     int *seg_ntile = reinterpret_cast<int *>(smem + L::kMisc + 16);
     int *seg_len = seg_ntile + SR_MAX_SEG;
     int *seg_start = seg_len + SR_MAX_SEG;
+    int *walk_start = seg_start + SR_MAX_SEG;   // (segment, tile) of this item's first tile
     float *row_alpha = reinterpret_cast<float *>(smem + L::kRow);   // [2][128]
     float *row_l = row_alpha + kQTiles * kTileM;                     // [2][128]
     float *row_m = row_l + kQTiles * kTileM;                         // [2][128]
@@ -161,6 +188,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&alpha_ready[t], 4);   // the four softmax warps of tile t
             mbar_init(&p_full[t], 8);        // four softmax + four correction warps
             mbar_init(&o_done[t], 1);
+            mbar_init(&stats_ready[t], 4);
         }
         *abort_flag = 0;
         int total = 0;
@@ -173,7 +201,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             seg_start[s] = p.seg_start[s];
             total += seg_ntile[s];
         }
-        *n_tiles_s = total;
+        // this item's share of the valid tiles, and where its walk starts
+        const int tile0 = static_cast<int>((static_cast<int64_t>(part) * total) / split);
+        const int tile1 = static_cast<int>((static_cast<int64_t>(part + 1) * total) / split);
+        int s0 = 0, k = tile0;
+        while (s0 < p.n_seg && (seg_ntile[s0] == 0 || k >= seg_ntile[s0])) {
+            k -= seg_ntile[s0];
+            ++s0;
+        }
+        n_tiles_s[0] = tile1 - tile0;
+        walk_start[0] = s0;
+        walk_start[1] = k;
         fence_mbarrier_init();
     }
     if (warp == kWarpMma) {
@@ -199,7 +237,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
         TileWalk w;
-        w.first(seg_ntile, n_seg);
+        w.s = walk_start[0];
+                w.t = walk_start[1];
         for (int j = 0; j < n_tiles; ++j, w.next(seg_ntile, n_seg)) {
             const int valid = min(kTileN, seg_len[w.s] - w.t * kTileN);
             if (!(ok = warp_wait(&s_full[t], j & 1, abort_flag, p.status))) break;
@@ -257,11 +296,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(&p_full[t]);
             }
         }
-        // hand the row statistics to the epilogue (one more alpha_ready phase)
+        // hand the row statistics to the epilogue
         row_l[t * kTileM + row] = l_run;
         row_m[t * kTileM + row] = m_run;
         __syncwarp();
-        if (ok && lane == 0) mbar_arrive(&alpha_ready[t]);
+        if (ok && lane == 0) mbar_arrive(&stats_ready[t]);
     } else if (warp < 4 * kQTiles + 4) {
         // ================================================================ correction + epilogue
         regs_decrease<kRegCorrection>();
@@ -299,44 +338,78 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         // ---------------------------------------------------------------- epilogue
+        if (split == 1) {
 #pragma unroll
-        for (int t = 0; t < kQTiles; ++t) {
-            const int grow = q0 + t * kTileM + row;
-            const bool row_ok = grow < q_len;
-            __nv_bfloat16 *orow = p.o + ((static_cast<size_t>(b) * p.q_cap + grow) * p.n_heads + h) * D;
-            if (n_tiles == 0) {
-                if (row_ok) {
-                    for (int d = 0; d < D; d += 8) *reinterpret_cast<uint4 *>(orow + d) = make_uint4(0, 0, 0, 0);
-                    if (p.lse) p.lse[static_cast<size_t>(bh) * p.q_cap + grow] = -INFINITY;
+            for (int t = 0; t < kQTiles; ++t) {
+                const int grow = q0 + t * kTileM + row;
+                const bool row_ok = grow < q_len;
+                __nv_bfloat16 *orow = p.o + ((static_cast<size_t>(b) * p.q_cap + grow) * p.n_heads + h) * D;
+                if (n_tiles == 0) {
+                    if (row_ok) {
+                        for (int d = 0; d < D; d += 8) *reinterpret_cast<uint4 *>(orow + d) = make_uint4(0, 0, 0, 0);
+                        if (p.lse) p.lse[static_cast<size_t>(bh) * p.q_cap + grow] = -INFINITY;
+                    }
+                    continue;
                 }
-                continue;
-            }
-            if (!ok) break;
-            if (!(ok = warp_wait(&alpha_ready[t], n_tiles & 1, abort_flag, p.status))) break;
-            if (!(ok = warp_wait(&o_done[t], (n_tiles - 1) & 1, abort_flag, p.status))) break;
-            tc_fence_after();
-            const float l_row = row_l[t * kTileM + row];
-            const float inv_l = 1.0f / l_row;
+                if (!ok) break;
+                if (!(ok = warp_wait(&stats_ready[t], 0, abort_flag, p.status))) break;
+                if (!(ok = warp_wait(&o_done[t], (n_tiles - 1) & 1, abort_flag, p.status))) break;
+                tc_fence_after();
+                const float l_row = row_l[t * kTileM + row];
+                const float inv_l = 1.0f / l_row;
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tmem + lane_base + tmem_o(t) + c * 32, r);
-                tmem_wait_ld();
-                if (row_ok) {
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem + lane_base + tmem_o(t) + c * 32, r);
+                    tmem_wait_ld();
+                    if (row_ok) {
 #pragma unroll
-                    for (int e = 0; e < 32; e += 8) {
-                        uint4 v;
-                        v.x = pack_bf16x2(__uint_as_float(r[e + 0]) * inv_l, __uint_as_float(r[e + 1]) * inv_l);
-                        v.y = pack_bf16x2(__uint_as_float(r[e + 2]) * inv_l, __uint_as_float(r[e + 3]) * inv_l);
-                        v.z = pack_bf16x2(__uint_as_float(r[e + 4]) * inv_l, __uint_as_float(r[e + 5]) * inv_l);
-                        v.w = pack_bf16x2(__uint_as_float(r[e + 6]) * inv_l, __uint_as_float(r[e + 7]) * inv_l);
-                        *reinterpret_cast<uint4 *>(orow + c * 32 + e) = v;
+                        for (int e = 0; e < 32; e += 8) {
+                            uint4 v;
+                            v.x = pack_bf16x2(__uint_as_float(r[e + 0]) * inv_l, __uint_as_float(r[e + 1]) * inv_l);
+                            v.y = pack_bf16x2(__uint_as_float(r[e + 2]) * inv_l, __uint_as_float(r[e + 3]) * inv_l);
+                            v.z = pack_bf16x2(__uint_as_float(r[e + 4]) * inv_l, __uint_as_float(r[e + 5]) * inv_l);
+                            v.w = pack_bf16x2(__uint_as_float(r[e + 6]) * inv_l, __uint_as_float(r[e + 7]) * inv_l);
+                            *reinterpret_cast<uint4 *>(orow + c * 32 + e) = v;
+                        }
                     }
                 }
+                if (row_ok && p.lse)
+                    p.lse[static_cast<size_t>(bh) * p.q_cap + grow] =
+                        (row_m[t * kTileM + row] + log2f(l_row)) * 0.69314718055994531f;
             }
-            if (row_ok && p.lse)
-                p.lse[static_cast<size_t>(bh) * p.q_cap + grow] =
-                    (row_m[t * kTileM + row] + log2f(l_row)) * 0.69314718055994531f;
+        } else {
+            // Split unit: publish this part's unnormalised (O, m, l); the
+            // combine kernel that follows on the stream merges the parts.
+            const int slot = item - p.n_full;
+            float *ws_m = p.ws_ml + static_cast<size_t>(slot) * 4 * kTileM;
+#pragma unroll 1
+            for (int t = 0; t < kQTiles; ++t) {
+                float *o_part =
+                    p.ws_o + (static_cast<size_t>(slot) * kQTiles + t) * kTileM * D + static_cast<size_t>(row) * D;
+                float m_part = -INFINITY, l_part = 0.f;
+                if (n_tiles > 0) {
+                    if (!ok) break;
+                    if (!(ok = warp_wait(&stats_ready[t], 0, abort_flag, p.status))) break;
+                    if (!(ok = warp_wait(&o_done[t], (n_tiles - 1) & 1, abort_flag, p.status))) break;
+                    tc_fence_after();
+                    m_part = row_m[t * kTileM + row];
+                    l_part = row_l[t * kTileM + row];
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t r[32];
+                        tmem_ld32(tmem + lane_base + tmem_o(t) + c * 32, r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; e += 4)
+                            __stcg(reinterpret_cast<float4 *>(o_part + c * 32 + e),
+                                   make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
+                                               __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3])));
+                    }
+                }
+                __stcg(ws_m + t * kTileM + row, m_part);
+                __stcg(ws_m + (2 + t) * kTileM + row, l_part);
+            }
         }
     } else {
         regs_decrease<kRegOther>();
@@ -354,7 +427,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tma_load_3d(smem + L::kQ + t * L::kTileBytes + pn * kPanelBytes, &tmQ, pn * 64,
                                     q0 + t * kTileM, bh, q_full);
                 TileWalk w;
-                w.first(seg_ntile, n_seg);
+                w.s = walk_start[0];
+                w.t = walk_start[1];
                 for (int j = 0; j < n_tiles; ++j, w.next(seg_ntile, n_seg)) {
                     const int st = j % kStages;
                     const uint32_t ph = (j / kStages) & 1;
@@ -442,6 +516,74 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// Merges the KV parts of every split unit: for each query row,
+//   M = max_q m_q,  L = sum_q l_q 2^(m_q - M),  O = sum_q 2^(m_q - M) O_q / L
+// (O_q unnormalised, m in log2 units).  One thread per (unit, row, 8 columns).
+struct CombineParams {
+    const float *ws_o;
+    const float *ws_ml;
+    __nv_bfloat16 *o;
+    float *lse;
+    const int32_t *q_len;
+    int32_t n_full, split, tail_units, qb_per_head, n_heads, q_cap;
+};
+
+template <int D>
+__global__ void __launch_bounds__(256) split_combine_kernel(const CombineParams c) {
+    constexpr int kChunks = D / 8;
+    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t total = static_cast<int64_t>(c.tail_units) * kQTiles * kTileM * kChunks;
+    if (idx >= total) return;
+    const int chunk = static_cast<int>(idx % kChunks);
+    const int r2 = static_cast<int>((idx / kChunks) % (kQTiles * kTileM));   // row within the 256-row block
+    const int tail = static_cast<int>(idx / (kChunks * kQTiles * kTileM));
+    const int t = r2 / kTileM, row = r2 % kTileM;
+    const int unit = c.n_full + tail;
+    const int qb = unit % c.qb_per_head, bh = unit / c.qb_per_head;
+    const int h = bh % c.n_heads, b = bh / c.n_heads;
+    const int grow = qb * kQTiles * kTileM + r2;
+    if (grow >= c.q_len[b]) return;
+    float mmax = -INFINITY;
+    for (int q = 0; q < c.split; ++q)
+        mmax = fmaxf(mmax, c.ws_ml[static_cast<size_t>(tail * c.split + q) * 4 * kTileM + t * kTileM + row]);
+    float lsum = 0.f, acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int q = 0; q < c.split; ++q) {
+        const float *mq = c.ws_ml + static_cast<size_t>(tail * c.split + q) * 4 * kTileM;
+        const float lq = mq[(2 + t) * kTileM + row];
+        if (!(lq > 0.f)) continue;
+        const float w = fast_exp2(mq[t * kTileM + row] - mmax);
+        lsum += lq * w;
+        const float *oq =
+            c.ws_o + (static_cast<size_t>(tail * c.split + q) * kQTiles + t) * kTileM * D + static_cast<size_t>(row) * D + chunk * 8;
+        const float4 x0 = *reinterpret_cast<const float4 *>(oq);
+        const float4 x1 = *reinterpret_cast<const float4 *>(oq + 4);
+        acc[0] += w * x0.x; acc[1] += w * x0.y; acc[2] += w * x0.z; acc[3] += w * x0.w;
+        acc[4] += w * x1.x; acc[5] += w * x1.y; acc[6] += w * x1.z; acc[7] += w * x1.w;
+    }
+    const float inv = lsum > 0.f ? 1.0f / lsum : 0.f;
+    uint4 v;
+    v.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+    v.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+    v.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
+    v.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+    *reinterpret_cast<uint4 *>(c.o + ((static_cast<size_t>(b) * c.q_cap + grow) * c.n_heads + h) * D + chunk * 8) = v;
+    if (chunk == 0 && c.lse)
+        c.lse[static_cast<size_t>(bh) * c.q_cap + grow] =
+            lsum > 0.f ? (mmax + log2f(lsum)) * 0.69314718055994531f : -INFINITY;
+}
+
+int sm_count() {
+    static int cached[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cached[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
 template <int D>
 int launch(const AttnLaunch &a) {
     using L = Smem<D>;
@@ -467,6 +609,20 @@ int launch(const AttnLaunch &a) {
     p.n_heads = a.n_heads;
     p.q_cap = a.q_cap;
     p.scale_log2 = static_cast<float>(static_cast<double>(a.softmax_scale) * 1.4426950408889634);
+    const AttnSchedule sc = attention_schedule(a.n_batch, a.n_heads, D, a.q_cap, sm_count());
+    p.qb_per_head = sc.qb_per_head;
+    p.n_full = sc.n_full;
+    p.split = 1;
+    int64_t items = sc.units;
+    if (sc.split > 1 && a.workspace && a.workspace_bytes >= sc.workspace_bytes) {
+        uint8_t *ws = static_cast<uint8_t *>(a.workspace);
+        p.split = sc.split;
+        p.ws_o = reinterpret_cast<float *>(ws);
+        p.ws_ml = reinterpret_cast<float *>(ws + sc.o_bytes);
+        items = sc.n_full + static_cast<int64_t>(sc.tail_units) * sc.split;
+    } else {
+        p.n_full = static_cast<int32_t>(sc.units);
+    }
     static bool attr_set[64] = {};   // the shared-memory opt-in is per device
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -476,14 +632,49 @@ int launch(const AttnLaunch &a) {
         if (e != cudaSuccess) return set_cuda_error("cudaFuncSetAttribute(chunk_attention)", e);
         if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
-    dim3 grid((a.q_cap + kQTiles * kTileM - 1) / (kQTiles * kTileM), a.n_heads, a.n_batch);
-    chunk_attention_kernel<D><<<grid, kThreads, L::kAlloc, a.stream>>>(tq, tk, tv, p);
+    if (items > 0x7fffffff) return set_error(SR_ERR_INVALID_ARG, "chunk_attention: too many work items");
+    chunk_attention_kernel<D><<<static_cast<unsigned>(items), kThreads, L::kAlloc, a.stream>>>(tq, tk, tv, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return set_cuda_error("chunk_attention launch", e);
+    if (p.split > 1) {
+        CombineParams c{p.ws_o, p.ws_ml, p.o, p.lse, p.q_len, p.n_full, p.split, sc.tail_units, p.qb_per_head,
+                        p.n_heads, p.q_cap};
+        const int64_t threads = static_cast<int64_t>(sc.tail_units) * kQTiles * kTileM * (D / 8);
+        split_combine_kernel<D><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, a.stream>>>(c);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return set_cuda_error("split_combine launch", e);
+    }
     return SR_OK;
 }
 
 }  // namespace
+
+AttnSchedule attention_schedule(int32_t n_batch, int32_t n_heads, int32_t head_dim, int32_t q_cap, int32_t sms) {
+    AttnSchedule sc{};
+    sc.qb_per_head = (q_cap + kQTiles * kTileM - 1) / (kQTiles * kTileM);
+    sc.units = static_cast<int64_t>(n_batch) * n_heads * sc.qb_per_head;
+    const int64_t P = sms > 0 ? sms : 148;
+    const int64_t full = (sc.units / P) * P;
+    const int64_t rem = sc.units - full;
+    sc.split = 1;
+    sc.n_full = static_cast<int32_t>(sc.units);
+    if (rem > 0) {
+        int64_t s = P / rem;
+        if (s > 8) s = 8;
+        if (s >= 2) {
+            sc.split = static_cast<int32_t>(s);
+            sc.n_full = static_cast<int32_t>(full);
+            sc.tail_units = static_cast<int32_t>(rem);
+        }
+    }
+    const int64_t slots = static_cast<int64_t>(sc.tail_units) * sc.split;
+    sc.o_bytes = static_cast<size_t>(slots) * kQTiles * kTileM * head_dim * sizeof(float);
+    sc.ml_bytes = static_cast<size_t>(slots) * 4 * kTileM * sizeof(float);
+    sc.workspace_bytes = sc.split > 1 ? sc.o_bytes + sc.ml_bytes : 0;
+    return sc;
+}
+
+int attention_sm_count() { return sm_count(); }
 
 int launch_chunk_attention(const AttnLaunch &a) {
     if (a.head_dim == 128) return launch<128>(a);

@@ -28,9 +28,25 @@ struct AttnLaunch {
     int32_t n_seg, n_batch, n_heads, head_dim, q_cap;
     int64_t kv_tokens;
     float softmax_scale;
+    void *workspace;
+    size_t workspace_bytes;
     cudaStream_t stream;
 };
 int launch_chunk_attention(const AttnLaunch &a);
+
+// Work list of the attention kernel: units are (session, head, 256-row query
+// block); whole waves of units run one per CTA, and the units of a last
+// partial wave are split into `split` KV ranges that fill the idle SMs.
+struct AttnSchedule {
+    int32_t qb_per_head;
+    int64_t units;
+    int32_t n_full;        // items that are whole units
+    int32_t split;         // parts per tail unit (1 = no split)
+    int32_t tail_units;
+    size_t o_bytes, ml_bytes, workspace_bytes;
+};
+AttnSchedule attention_schedule(int32_t n_batch, int32_t n_heads, int32_t head_dim, int32_t q_cap, int32_t sms);
+int attention_sm_count();
 
 struct RopeLaunch {
     const void *x;

@@ -151,6 +151,8 @@ class StreamingWindow:
         self.o = torch.zeros(B, self.q_cap, H, D, dtype=torch.bfloat16, **kw)
         self.lse = torch.zeros(B, H, self.q_cap, dtype=torch.float32, **kw)
         self.status = torch.zeros(1, dtype=torch.int32, **kw)
+        ws = capi.sr_chunk_attention_workspace_bytes(B, H, D, self.q_cap) if self.device.type == "cuda" else 0
+        self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, **kw) if ws else None
         lens = np.array([[p.lengths[s] for s in self.segments] for p in self.plans], dtype=np.int32)
         self.lengths = lens
         self.kv_len = torch.from_numpy(lens).to(self.device)
@@ -247,7 +249,7 @@ class StreamingWindow:
     def attend(self, stream=None) -> torch.Tensor:
         """a4: fused chunk attention -> o [B, q_cap, H, D] (and lse)."""
         capi.sr_chunk_attention_fwd(self.q_att, self.k_att, self.v, self.o, self.lse, self.caps, self.kv_len,
-                                    self.q_len, self.scale, self.status, stream=stream)
+                                    self.q_len, self.scale, self.status, workspace=self.workspace, stream=stream)
         return self.o
 
     def step(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream=None) -> torch.Tensor:

@@ -8,7 +8,7 @@ import pytest
 from streaming_video_audio_b200 import capi
 
 EXPECTED = {"sr_version", "sr_get_last_error", "sr_rope3d_apply", "sr_history_compress", "sr_kv_append",
-            "sr_chunk_attention_fwd"}
+            "sr_chunk_attention_fwd", "sr_chunk_attention_workspace_bytes"}
 
 
 def test_header_declares_the_boundary():
@@ -34,7 +34,7 @@ def test_attention_rejects_bad_arguments_on_host():
 
     def call(a):
         return lib.sr_chunk_attention_fwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["lay"], a["kl"], a["ql"],
-                                          a["B"], a["H"], a["D"], a["qcap"], a["scale"], None, None)
+                                          a["B"], a["H"], a["D"], a["qcap"], a["scale"], None, 0, None, None)
 
     assert call(args(D=96)) == capi.SR_ERR_UNSUPPORTED and "head_dim" in _err(lib)
     assert call(args(qcap=0)) == capi.SR_ERR_INVALID_ARG

@@ -163,14 +163,17 @@ def _draw_case(D, H, caps, lens, q_len, seed, perturb_padding=False):
     return q, k, v
 
 
-def _run_attention(q, k, v, caps, lens, q_len):
+def _run_attention(q, k, v, caps, lens, q_len, use_workspace=True):
     B, H, q_cap, D = q.shape
     o = torch.full((B, q_cap, H, D), 3.0, dtype=torch.bfloat16, device=DEV)
     lse = torch.zeros(B, H, q_cap, device=DEV)
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    nbytes = capi.sr_chunk_attention_workspace_bytes(B, H, D, q_cap)
+    ws = torch.full((max(nbytes, 16),), 0xAB, dtype=torch.uint8, device=DEV) if use_workspace and nbytes else None
     capi.sr_chunk_attention_fwd(q.to(DEV).contiguous(), k.to(DEV).contiguous(), v.to(DEV).contiguous(), o, lse,
                                 caps, torch.tensor(lens, dtype=torch.int32, device=DEV),
-                                torch.tensor(q_len, dtype=torch.int32, device=DEV), 1 / math.sqrt(D), status)
+                                torch.tensor(q_len, dtype=torch.int32, device=DEV), 1 / math.sqrt(D), status,
+                                workspace=ws)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     return o.cpu(), lse.cpu()
@@ -227,3 +230,42 @@ def test_attention_all_segments_empty_writes_zeros():
     D, H, caps = 64, 1, [128, 128]
     _, _, _, o, lse = _attention_case(D, H, caps, [[0, 0]], [5], seed=40)
     assert torch.all(o[0, :5] == 0) and torch.all(torch.isinf(lse[0, 0, :5]))
+
+
+def test_attention_split_schedule_matches_whole_units():
+    """With a workspace the last partial wave is split along the KV tiles and
+    merged in fp32; without one every unit runs whole.  Both are checked
+    against the oracle and against each other."""
+    D, H, caps = 128, 5, [256, 1024, 384]
+    lens = [[256, 1000, 300]]
+    q_len = [700]
+    nbytes = capi.sr_chunk_attention_workspace_bytes(1, H, D, 700)
+    assert nbytes > 0   # 5 heads x 3 query blocks < one wave: split is active
+    q, k, v = _draw_case(D, H, caps, lens, q_len, seed=50)
+    o_split, l_split = _run_attention(q, k, v, caps, lens, q_len, use_workspace=True)
+    o_whole, l_whole = _run_attention(q, k, v, caps, lens, q_len, use_workspace=False)
+    assert float((o_split[0, :700].float() - o_whole[0, :700].float()).abs().max()) <= 2 ** -7
+    assert float((l_split[0, :, :700] - l_whole[0, :, :700]).abs().max()) <= 1e-4
+    for h in range(H):
+        kk, vv = _valid_kv(k, v, 0, h, caps, lens[0])
+        ro, rl = oracle.attention(q[0, h, :700], kk, vv, 1 / math.sqrt(D))
+        for o_ in (o_split, o_whole):
+            mx, mean = attn_errors(o_[0, :700, h], ro)
+            assert mx <= ATTN_MAX_ABS and mean <= ATTN_MEAN_ABS
+
+
+def test_attention_repeated_launches_deterministic():
+    """Many launches of ragged, few-tile work (split parts of one or two tiles,
+    empty parts, empty segments): no pipeline wait may give up and every
+    launch must produce the same bits."""
+    D, H, caps = 128, 3, [128, 1024, 256]
+    lens = [[1, 1000, 129], [128, 7, 256], [0, 513, 255]]
+    q_len = [129, 256, 255]
+    q, k, v = _draw_case(D, H, caps, lens, q_len, seed=60)
+    o0, l0 = _run_attention(q, k, v, caps, lens, q_len)
+    for _ in range(40):
+        o, l = _run_attention(q, k, v, caps, lens, q_len)
+        assert torch.equal(o, o0) and torch.equal(l, l0)
+    for _ in range(10):
+        o, l = _run_attention(q, k, v, caps, lens, q_len, use_workspace=False)
+        assert torch.equal(o[0, :129], _run_attention(q, k, v, caps, lens, q_len, use_workspace=False)[0][0, :129])
