@@ -222,6 +222,38 @@ int sr_chunk_attention_fwd(const void *q, const void *k, const void *v, void *o,
  * only; reads the device's SM count (no allocation, no synchronisation). */
 size_t sr_chunk_attention_workspace_bytes(int32_t n_batch, int32_t n_heads, int32_t head_dim, int32_t q_cap);
 
+/* Allocation-free variant of sr_chunk_attention_fwd (the pages have no
+ * counterpart; this is a packaging option of this library).
+ *
+ * For callers that cannot allocate device memory when they run the
+ * attention -- a plugin inside another runtime that only receives its input
+ * and output buffers, a real-time frame loop where cudaMalloc (which may
+ * synchronise the device) is not allowed, or an application whose device
+ * memory is all owned by its own allocator.  Arguments, layouts and results
+ * are those of sr_chunk_attention_fwd; the split-KV scratch comes from a
+ * static device array of SR_NOALLOC_SCRATCH_BYTES (24 MiB) that every GPU
+ * loading the library holds until the process exits.  The call allocates
+ * nothing and frees nothing.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Problems whose schedule needs more scratch than the array holds
+ *     (sr_chunk_attention_workspace_bytes > SR_NOALLOC_SCRATCH_BYTES) are
+ *     rejected with SR_ERR_UNSUPPORTED and nothing is launched.  On a 148-SM
+ *     B200 the largest need is about 19.7 MB, so no problem is rejected there.
+ *   - All calls on a device share the array and it keeps the last call's
+ *     contents; nothing in it needs to start at zero.  Calls that could
+ *     execute concurrently on the same device (different streams or host
+ *     threads) race on it: order them.
+ */
+#define SR_NOALLOC_SCRATCH_BYTES (24u * 1024u * 1024u)
+
+int sr_chunk_attention_fwd_noalloc(const void *q, const void *k, const void *v, void *o, float *lse,
+                                   const sr_kv_layout *layout, const int32_t *kv_len_dev,
+                                   const int32_t *q_len_dev, int32_t n_batch, int32_t n_heads,
+                                   int32_t head_dim, int32_t q_cap, float softmax_scale,
+                                   int32_t *status_dev, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -277,3 +277,49 @@ def sr_chunk_attention_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o:
     _check("sr_chunk_attention_fwd", load().sr_chunk_attention_fwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), ctypes.byref(lay), _ptr(kv_len), _ptr(q_len),
         B, H, D, q_cap, float(softmax_scale), _ptr(workspace), ws_bytes, _ptr(status), _stream(stream)))
+
+
+SR_NOALLOC_SCRATCH_BYTES = 24 * 1024 * 1024
+
+
+def sr_chunk_attention_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+                                   lse: Optional[torch.Tensor], caps: Sequence[int], kv_len: torch.Tensor,
+                                   q_len: torch.Tensor, softmax_scale: float, status: Optional[torch.Tensor] = None,
+                                   stream=None) -> None:
+    """The attention for callers that cannot allocate device memory while they
+    run it (a plugin handed only its inputs and outputs, a real-time loop that
+    must not call cudaMalloc, an application whose memory belongs to its own
+    allocator): same arguments and results as sr_chunk_attention_fwd, with the
+    split-KV scratch taken from the library's static 24 MiB device array.  The
+    first call on a device resolves that array's address, so make it before
+    any stream capture; calls that may overlap on one device must be ordered,
+    since they share the array."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _cuda(t, torch.bfloat16, n)
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    _cuda(lse, torch.float32, "lse")
+    _cuda(kv_len, torch.int32, "kv_len")
+    _cuda(q_len, torch.int32, "q_len")
+    _cuda(status, torch.int32, "status")
+    B, H, q_cap, D = q.shape
+    kv_tokens = int(sum(caps))
+    if tuple(k.shape) != (B, H, kv_tokens, D) or tuple(v.shape) != (B, H, kv_tokens, D):
+        raise ValueError("k and v must be [B, H, sum(caps), D]")
+    if tuple(o.shape) != (B, q_cap, H, D):
+        raise ValueError("o must be [B, q_cap, H, D]")
+    if lse is not None and (tuple(lse.shape) != (B, H, q_cap) or not lse.is_contiguous()):
+        raise ValueError("lse must be contiguous [B, H, q_cap]")
+    if tuple(kv_len.shape) != (B, len(caps)) or not kv_len.is_contiguous():
+        raise ValueError("kv_len must be contiguous int32 [B, n_seg]")
+    if tuple(q_len.shape) != (B,) or not q_len.is_contiguous():
+        raise ValueError("q_len must be contiguous int32 [B]")
+    lib = load()
+    fn = lib.sr_chunk_attention_fwd_noalloc
+    fn.argtypes = [_vp, _vp, _vp, _vp, _vp, ctypes.POINTER(sr_kv_layout), _vp, _vp, _i32, _i32, _i32, _i32, _f32,
+                   _vp, _vp]
+    fn.restype = ctypes.c_int
+    lay = make_layout(caps)
+    _check("sr_chunk_attention_fwd_noalloc", fn(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), ctypes.byref(lay), _ptr(kv_len), _ptr(q_len),
+        B, H, D, q_cap, float(softmax_scale), _ptr(status), _stream(stream)))

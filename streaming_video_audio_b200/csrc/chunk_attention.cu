@@ -33,6 +33,8 @@
 // aliases the first 64 columns of S_t.  Every wait is bounded
 // (sr_device.cuh): a stuck pipeline sets the status word and the CTA returns
 // instead of hanging.
+#include <mutex>
+
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -682,4 +684,65 @@ int launch_chunk_attention(const AttnLaunch &a) {
     return set_error(SR_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
 }
 
+// ============================================================================
+// Allocation-free variant of sr_chunk_attention_fwd.
+//
+// Some callers cannot allocate device memory at the moment they run the
+// attention: a plugin living inside another runtime that is handed only its
+// input and output buffers, a real-time frame loop in which cudaMalloc (which
+// may synchronise the whole device) is forbidden, or an application whose
+// device memory is entirely owned by its own allocator.  For them the scratch
+// that the split-KV schedule needs lives in this file-scope device array,
+// which exists once per GPU that loads the library and stays there until the
+// process exits.  Nothing in it has to start at zero: every partial result the
+// merge step reads is written earlier in the same call.  All calls on a device
+// share it, so calls that could run at the same time on that device (other
+// streams, other host threads) race and must be ordered by the caller.
+namespace {
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[SR_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mutex;
+void *g_noalloc_ptr[64] = {};   // device address of g_noalloc_scratch, per device
+
+// Device address of the scratch array on the current device.  The host-side
+// name g_noalloc_scratch is only a stand-in for the symbol; the address a
+// kernel may use comes from cudaGetSymbolAddress, resolved once per device
+// with that device current.
+int noalloc_scratch(void **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return set_cuda_error("cudaGetDevice", e);
+    if (dev < 0 || dev >= 64) return set_error(SR_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+    std::lock_guard<std::mutex> guard(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void *ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (e != cudaSuccess) return set_cuda_error("cudaGetSymbolAddress(static attention scratch)", e);
+        g_noalloc_ptr[dev] = ptr;
+    }
+    *out = g_noalloc_ptr[dev];
+    return SR_OK;
+}
+
+}  // namespace
+
 }  // namespace sr
+
+extern "C" int sr_chunk_attention_fwd_noalloc(const void *q, const void *k, const void *v, void *o, float *lse,
+                                               const sr_kv_layout *layout, const int32_t *kv_len_dev,
+                                               const int32_t *q_len_dev, int32_t n_batch, int32_t n_heads,
+                                               int32_t head_dim, int32_t q_cap, float softmax_scale,
+                                               int32_t *status_dev, void *stream) {
+    const size_t need = sr_chunk_attention_workspace_bytes(n_batch, n_heads, head_dim, q_cap);
+    if (need > SR_NOALLOC_SCRATCH_BYTES)
+        return sr::set_error(SR_ERR_UNSUPPORTED,
+                             "chunk_attention_noalloc: this problem needs %zu bytes of scratch, the static scratch "
+                             "holds %zu",
+                             need, static_cast<size_t>(SR_NOALLOC_SCRATCH_BYTES));
+    void *scratch = nullptr;
+    const int rc = sr::noalloc_scratch(&scratch);
+    if (rc != SR_OK) return rc;
+    return sr_chunk_attention_fwd(q, k, v, o, lse, layout, kv_len_dev, q_len_dev, n_batch, n_heads, head_dim, q_cap,
+                                  softmax_scale, scratch, SR_NOALLOC_SCRATCH_BYTES, status_dev, stream);
+}
