@@ -20,8 +20,12 @@
 //               back into TMEM over the S columns.  The max only moves when it
 //               grows by more than 2^8 (lazy rescale: exact, the final
 //               normalisation uses the same stale max).
-//   warps 8-11  correction: rescale O_t in TMEM when a row's max moved, and the
-//               epilogue (O / l -> bf16 token-major, LSE).
+//               When a row's max does move, the softmax warp rescales its O_t
+//               row in TMEM itself: S_t(j) is issued after PV_t(j-1) and its
+//               commit tracks every earlier MMA, so once S_t(j) has landed
+//               PV_t(j-1) has too, and PV_t(j) waits for this warp's P.
+//   warps 8-11  epilogue: O / l -> bf16 token-major output and LSE (or the
+//               unnormalised partials of a split unit).
 //   warp 12     TMA producer: Q0, Q1 once, then K and V tiles (128 tokens) into
 //               two-stage rings, walking only the segments' valid tiles.
 //   warp 13     TMEM owner + single-thread tcgen05.mma issuer, ping-pong order
@@ -55,6 +59,7 @@ constexpr int kWarpTma = 12, kWarpMma = 13;
 constexpr int kPanelBytes = 128 * 128;   // 128 rows x 128 bytes (64 bf16), one swizzle-128B panel
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
+
 // Registers per thread after reallocation (launch: 65536 / 512 = 128 each):
 // 2 x 128 x 160 + 128 x 88 + 128 x 104 = 65536 (the launch total; no spills).
 constexpr int kRegSoftmax = 160, kRegCorrection = 88, kRegOther = 104;
@@ -93,22 +98,17 @@ struct Smem {
     static constexpr int kV = kK + kStages * kTileBytes;
     static constexpr int kBar = kV + kStages * kTileBytes;
     // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S],
-    // s_full[2], alpha_ready[2], p_full[2], o_done[2], stats_ready[2]
-    static constexpr int kNumBars = 1 + 4 * kStages + 5 * kQTiles;
+    // s_full[2], p_full[2], o_done[2], stats_ready[2]
+    static constexpr int kNumBars = 1 + 4 * kStages + 4 * kQTiles;
     static constexpr int kMisc = kBar + kNumBars * 8;
-    static constexpr int kRow = kMisc + 16 + 12 * SR_MAX_SEG + 16;   // float alpha[2][128], l[2][128], m[2][128]
-    static constexpr int kEnd = kRow + 3 * kQTiles * kTileM * 4;
+    static constexpr int kRow = kMisc + 16 + 12 * SR_MAX_SEG + 16;   // float l[2][128], m[2][128]
+    static constexpr int kEnd = kRow + 2 * kQTiles * kTileM * 4;
     static constexpr int kAlloc = kEnd + 1024;   // slack for manual 1024-byte alignment
 };
 
 // Walks the valid 128-token tiles of every segment in buffer order.
 struct TileWalk {
     int s, t;
-    __device__ void first(const int *ntile, int n_seg) {
-        s = 0;
-        t = 0;
-        while (s < n_seg && ntile[s] == 0) ++s;
-    }
     __device__ void next(const int *ntile, int n_seg) {
         if (++t == ntile[s]) {
             t = 0;
@@ -157,13 +157,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *v_full = k_empty + kStages;
     uint64_t *v_empty = v_full + kStages;
     uint64_t *s_full = v_empty + kStages;        // [2] MMA -> softmax t
-    uint64_t *alpha_ready = s_full + kQTiles;    // [2] softmax t -> correction
-    uint64_t *p_full = alpha_ready + kQTiles;    // [2] softmax t + correction -> MMA
-    uint64_t *o_done = p_full + kQTiles;         // [2] MMA (PV_t) -> correction
-    // [2] softmax t -> epilogue: final row max / sum.  A barrier of its own:
-    // a second arrival on alpha_ready could complete two phases before the
-    // correction warps wait on the first, and parity waits would alias.
-    uint64_t *stats_ready = o_done + kQTiles;
+    uint64_t *p_full = s_full + kQTiles;         // [2] softmax t -> MMA (P_t written, O_t rescaled)
+    uint64_t *o_done = p_full + kQTiles;         // [2] MMA (PV_t) -> epilogue
+    uint64_t *stats_ready = o_done + kQTiles;    // [2] softmax t -> epilogue: final row max / sum
+    // Every waiter consumes each phase of its barrier in order, so parity
+    // waits never alias: a barrier is never more than one phase ahead of the
+    // phase its waiter asks for.
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
     int *n_tiles_s = reinterpret_cast<int *>(smem + L::kMisc + 8);
@@ -171,9 +170,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int *seg_len = seg_ntile + SR_MAX_SEG;
     int *seg_start = seg_len + SR_MAX_SEG;
     int *walk_start = seg_start + SR_MAX_SEG;   // (segment, tile) of this item's first tile
-    float *row_alpha = reinterpret_cast<float *>(smem + L::kRow);   // [2][128]
-    float *row_l = row_alpha + kQTiles * kTileM;                     // [2][128]
-    float *row_m = row_l + kQTiles * kTileM;                         // [2][128]
+    float *row_l = reinterpret_cast<float *>(smem + L::kRow);   // [2][128]
+    float *row_m = row_l + kQTiles * kTileM;                     // [2][128]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -187,8 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int t = 0; t < kQTiles; ++t) {
             mbar_init(&s_full[t], 1);
-            mbar_init(&alpha_ready[t], 4);   // the four softmax warps of tile t
-            mbar_init(&p_full[t], 8);        // four softmax + four correction warps
+            mbar_init(&p_full[t], 4);        // the four softmax warps of tile t
             mbar_init(&o_done[t], 1);
             mbar_init(&stats_ready[t], 4);
         }
@@ -240,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         TileWalk w;
         w.s = walk_start[0];
-                w.t = walk_start[1];
+        w.t = walk_start[1];
         for (int j = 0; j < n_tiles; ++j, w.next(seg_ntile, n_seg)) {
             const int valid = min(kTileN, seg_len[w.s] - w.t * kTileN);
             if (!(ok = warp_wait(&s_full[t], j & 1, abort_flag, p.status))) break;
@@ -260,12 +257,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int c = 0; c < kTileN; ++c) s[c] = c < valid ? s[c] : -INFINITY;
             }
-            // row max: eight independent chains, then a tree
+            // row max over eight independent chains, then a tree
             float mx8[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) mx8[i] = s[i];
 #pragma unroll
-            for (int c = 8; c < kTileN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+            for (int c = 8; c < kTileN; c += 16)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) mx8[i] = fmax3(mx8[i], s[c + i], s[c + 8 + i]);
             const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                    fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
             const float m_new = fmaxf(m_run, mx * sl2);
@@ -281,7 +280,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
             l_run = l_run * alpha + sum;
             m_run = m_use;
-            row_alpha[t * kTileM + row] = alpha;
             // P (bf16 pairs) over the first 64 columns of S_t
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
@@ -290,13 +288,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(s[half * 64 + 2 * e], s[half * 64 + 2 * e + 1]);
                 tmem_st32(s_addr + half * 32, pk);
             }
+            if (j > 0 && __any_sync(0xffffffffu, need)) {
+                // PV_t(j-1) is complete (see the design note); PV_t(j) waits for us
+                const uint32_t o_addr = tmem + lane_base + tmem_o(t);
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(o_addr + c * 32, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+                    tmem_st32(o_addr + c * 32, r);
+                }
+            }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&alpha_ready[t]);
-                mbar_arrive(&p_full[t]);
-            }
+            if (lane == 0) mbar_arrive(&p_full[t]);
         }
         // hand the row statistics to the epilogue
         row_l[t * kTileM + row] = l_run;
@@ -304,41 +312,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (ok && lane == 0) mbar_arrive(&stats_ready[t]);
     } else if (warp < 4 * kQTiles + 4) {
-        // ================================================================ correction + epilogue
+        // ================================================================ epilogue
         regs_decrease<kRegCorrection>();
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
         bool ok = true;
-        for (int j = 0; ok && j < n_tiles; ++j) {
-#pragma unroll
-            for (int t = 0; t < kQTiles; ++t) {
-                if (!(ok = warp_wait(&alpha_ready[t], j & 1, abort_flag, p.status))) break;
-                const float alpha = row_alpha[t * kTileM + row];
-                if (j > 0) {
-                    // PV_t(j-1) must have landed before O_t is touched; waiting on
-                    // every phase also keeps the parity waits from lagging.
-                    if (!(ok = warp_wait(&o_done[t], (j - 1) & 1, abort_flag, p.status))) break;
-                    if (__any_sync(0xffffffffu, alpha != 1.0f)) {
-                        tc_fence_after();
-#pragma unroll
-                        for (int c = 0; c < D / 32; ++c) {
-                            uint32_t r[32];
-                            const uint32_t o_addr = tmem + lane_base + tmem_o(t) + c * 32;
-                            tmem_ld32(o_addr, r);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-                            tmem_st32(o_addr, r);
-                        }
-                        tmem_wait_st();
-                    }
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&p_full[t]);
-            }
-        }
         // ---------------------------------------------------------------- epilogue
         if (split == 1) {
 #pragma unroll

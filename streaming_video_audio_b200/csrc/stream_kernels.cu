@@ -41,7 +41,7 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
 // computed on the host in double.
 struct RopeTable {
     double theta[64];
-    int8_t axis[64];
+    int32_t pairs_t, pairs_th;   // pairs of the t block, of the t and h blocks together
 };
 
 struct RopeArgs {
@@ -55,19 +55,35 @@ struct RopeArgs {
 };
 
 // One CTA per (token, batch).  Thread t handles the 16-byte chunk
-// c = t % (D/8) of heads t/(D/8), t/(D/8) + 128/(D/8), ...: the angles of a
-// token depend on (token, pair) only, so each thread evaluates its four
-// (cos, sin) pairs once, in double precision (angle error independent of
-// the position's magnitude), and reuses them across all heads; the rotation
-// itself runs in fp32.
+// c = t % (D/8) of heads t/(D/8), t/(D/8) + 128/(D/8), ...  It first issues
+// the loads of all its heads (up to kIters of them in flight), then derives
+// the token's four (cos, sin) pairs -- they depend on (token, pair) only and
+// are reused for every head -- and finally rotates and stores.  The angle
+// p * theta is formed in double and reduced to [-pi, pi] in double, so its
+// error does not grow with the position's magnitude; the small remainder goes
+// through fp32 sincosf.  The rotation itself runs in fp32.
 template <int D>
 __global__ void __launch_bounds__(128) rope3d_kernel(const RopeArgs a, const RopeTable tab) {
     constexpr int kChunks = D / 8;
     constexpr int kHeadsPerPass = 128 / kChunks;
+    constexpr int kIters = 8;   // heads kept in flight per thread: 8 x 8 = 64 heads at D = 128
     const int n = blockIdx.x, b = blockIdx.y;
-    if (a.n_valid && n >= a.n_valid[b]) return;
+    if (a.n_valid && n >= a.n_valid[b]) return;   // uniform per CTA (before the barrier below)
     const int c = threadIdx.x % kChunks;
     const int hp = threadIdx.x / kChunks;
+    const __nv_bfloat16 *xt = a.x + b * a.xb + n * a.xt + c * 8;
+    __nv_bfloat16 *yt = a.y + b * a.yb + n * a.yt + c * 8;
+    uint4 u[kIters];
+#pragma unroll
+    for (int i = 0; i < kIters; ++i) {
+        const int h = hp + i * kHeadsPerPass;
+        if (h < a.n_heads) u[i] = __ldg(reinterpret_cast<const uint4 *>(xt + h * a.xh));
+    }
+    // theta per pair, staged once per CTA: indexing the parameter table with a
+    // per-thread index would serialise the constant-cache reads
+    __shared__ double s_theta[D / 2];
+    if (threadIdx.x < D / 2) s_theta[threadIdx.x] = tab.theta[threadIdx.x];
+    __syncthreads();
     float cs[4], sn[4];
     float pt = 0.f, ph = 0.f, pw = 0.f;
     if (a.pos) {
@@ -76,23 +92,36 @@ __global__ void __launch_bounds__(128) rope3d_kernel(const RopeArgs a, const Rop
         ph = pp[1];
         pw = pp[2];
     }
+    constexpr double kTwoPi = 6.283185307179586476925286766559;
+    constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         const int pair = c * 4 + k;
-        const int ax = tab.axis[pair];
-        const double pa = ax == 0 ? pt : (ax == 1 ? ph : pw);
-        double s, co;
-        sincos(pa * tab.theta[pair], &s, &co);
-        cs[k] = static_cast<float>(co * a.out_scale);
-        sn[k] = static_cast<float>(s * a.out_scale);
+        const double pa = pair < tab.pairs_t ? pt : (pair < tab.pairs_th ? ph : pw);
+        const double phi = pa * s_theta[pair];
+        const double r = fma(-rint(phi * kInvTwoPi), kTwoPi, phi);
+        float s, co;
+        sincosf(static_cast<float>(r), &s, &co);
+        cs[k] = co * a.out_scale;
+        sn[k] = s * a.out_scale;
     }
-    const __nv_bfloat16 *xt = a.x + b * a.xb + n * a.xt + c * 8;
-    __nv_bfloat16 *yt = a.y + b * a.yb + n * a.yt + c * 8;
-#pragma unroll 4
-    for (int h = hp; h < a.n_heads; h += kHeadsPerPass) {
-        const uint4 u = __ldg(reinterpret_cast<const uint4 *>(xt + h * a.xh));
+#pragma unroll
+    for (int i = 0; i < kIters; ++i) {
+        const int h = hp + i * kHeadsPerPass;
+        if (h < a.n_heads) {
+            float f[8], g[8];
+            unpack8(u[i], f);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                g[2 * k] = f[2 * k] * cs[k] - f[2 * k + 1] * sn[k];
+                g[2 * k + 1] = f[2 * k] * sn[k] + f[2 * k + 1] * cs[k];
+            }
+            *reinterpret_cast<uint4 *>(yt + h * a.yh) = pack8(g);
+        }
+    }
+    for (int h = hp + kIters * kHeadsPerPass; h < a.n_heads; h += kHeadsPerPass) {   // very many heads
         float f[8], g[8];
-        unpack8(u, f);
+        unpack8(__ldg(reinterpret_cast<const uint4 *>(xt + h * a.xh)), f);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             g[2 * k] = f[2 * k] * cs[k] - f[2 * k + 1] * sn[k];
@@ -113,28 +142,28 @@ struct PoolArgs {
     const float *__restrict__ frame_t;
     float *__restrict__ pos_out;
     int64_t pos_b;
-    int64_t total;   // threads doing work
+    int64_t total;   // threads doing work per (batch, frame)
 };
 
 // One thread per (batch, frame, cell, head, 16-byte chunk); chunk fastest so a
-// warp reads whole 256-byte head rows of each member token.
-template <int D>
+// warp reads whole 256-byte head rows of each member token.  PH, PW > 0 fix
+// the window at compile time so that all member loads of a tensor are in
+// flight together (members outside the grid are skipped); PH = PW = 0 reads
+// the window from the arguments.
+template <int D, int PH, int PW>
 __global__ void __launch_bounds__(256) pool_kernel(const PoolArgs a) {
     constexpr int kChunks = D / 8;
-    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (idx >= a.total) return;
-    int64_t rest = idx;
-    const int c = static_cast<int>(rest % kChunks);
-    rest /= kChunks;
-    const int h = static_cast<int>(rest % a.n_heads);
-    rest /= a.n_heads;
-    const int j = static_cast<int>(rest % a.cells);
-    rest /= a.cells;
-    const int f = static_cast<int>(rest % a.n_frames);
-    const int b = static_cast<int>(rest / a.n_frames);
+    const uint32_t idx = blockIdx.x * blockDim.x + threadIdx.x;   // (cell, head, chunk) of one frame
+    if (idx >= static_cast<uint32_t>(a.total)) return;
+    const int f = blockIdx.y, b = blockIdx.z;
+    const int c = static_cast<int>(idx % kChunks);
+    const uint32_t hj = idx / kChunks;
+    const int h = static_cast<int>(hj % static_cast<uint32_t>(a.n_heads));
+    const int j = static_cast<int>(hj / static_cast<uint32_t>(a.n_heads));
+    const int ph = PH > 0 ? PH : a.pool_h, pw = PW > 0 ? PW : a.pool_w;
     const int r = j / a.cells_w, cc = j % a.cells_w;
-    const int r0 = r * a.pool_h, r1 = min(r0 + a.pool_h, a.grid_h);
-    const int c0 = cc * a.pool_w, c1 = min(c0 + a.pool_w, a.grid_w);
+    const int r0 = r * ph, r1 = min(r0 + ph, a.grid_h);
+    const int c0 = cc * pw, c1 = min(c0 + pw, a.grid_w);
     const float count = static_cast<float>((r1 - r0) * (c1 - c0));
     const int64_t in_off = b * a.ib + f * a.i_f + h * a.ih + c * 8;
     const int64_t out_off = b * a.ob + f * a.o_f + j * a.ot + h * a.oh + c * 8;
@@ -144,15 +173,34 @@ __global__ void __launch_bounds__(256) pool_kernel(const PoolArgs a) {
         __nv_bfloat16 *dst = which ? a.v_out : a.k_out;
         if (!src) continue;
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int rr = r0; rr < r1; ++rr) {
-#pragma unroll 4
-            for (int ci = c0; ci < c1; ++ci) {
-                const uint4 u = __ldg(reinterpret_cast<const uint4 *>(
-                    src + in_off + static_cast<int64_t>(rr * a.grid_w + ci) * a.it));
+        if constexpr (PH > 0 && PW > 0) {
+            uint4 u[PH * PW];
+#pragma unroll
+            for (int m = 0; m < PH * PW; ++m) {
+                const int rr = r0 + m / PW, ci = c0 + m % PW;
+                u[m] = (rr < r1 && ci < c1)
+                           ? __ldg(reinterpret_cast<const uint4 *>(src + in_off +
+                                                                   static_cast<int64_t>(rr * a.grid_w + ci) * a.it))
+                           : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int m = 0; m < PH * PW; ++m) {
                 float v[8];
-                unpack8(u, v);
+                unpack8(u[m], v);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) acc[e] += v[e];
+            }
+        } else {
+            for (int rr = r0; rr < r1; ++rr) {
+#pragma unroll 4
+                for (int ci = c0; ci < c1; ++ci) {
+                    const uint4 u = __ldg(reinterpret_cast<const uint4 *>(
+                        src + in_off + static_cast<int64_t>(rr * a.grid_w + ci) * a.it));
+                    float v[8];
+                    unpack8(u, v);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) acc[e] += v[e];
+                }
             }
         }
 #pragma unroll
@@ -198,15 +246,13 @@ struct AppendArgs {
 template <int D>
 __global__ void __launch_bounds__(256) append_kernel(const AppendArgs a) {
     constexpr int kChunks = D / 8;
-    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (idx >= a.total) return;
-    int64_t rest = idx;
-    const int c = static_cast<int>(rest % kChunks);
-    rest /= kChunks;
-    const int h = static_cast<int>(rest % a.n_heads);
-    rest /= a.n_heads;
-    const int n = static_cast<int>(rest % a.n_tokens);
-    const int b = static_cast<int>(rest / a.n_tokens);
+    const uint32_t idx = blockIdx.x * blockDim.x + threadIdx.x;   // (token, head, chunk) of one session
+    if (idx >= static_cast<uint32_t>(a.total)) return;
+    const int b = blockIdx.y;
+    const int c = static_cast<int>(idx % kChunks);
+    const uint32_t hn = idx / kChunks;
+    const int h = static_cast<int>(hn % static_cast<uint32_t>(a.n_heads));
+    const int n = static_cast<int>(hn / static_cast<uint32_t>(a.n_heads));
     if (a.n_valid && n >= a.n_valid[b]) return;
     const int64_t s_off = b * a.sb + n * a.st + h * a.sh + c * 8;
     const int64_t d_off =
@@ -230,10 +276,10 @@ int rope_launch(const RopeLaunch &l) {
     const int widths[3] = {l.cfg.d_t, l.cfg.d_h, l.cfg.d_w};
     int pair = 0;
     for (int ax = 0; ax < 3; ++ax)
-        for (int j = 0; j < widths[ax] / 2; ++j, ++pair) {
-            tab.axis[pair] = static_cast<int8_t>(ax);
+        for (int j = 0; j < widths[ax] / 2; ++j, ++pair)
             tab.theta[pair] = std::pow(static_cast<double>(l.cfg.base), -2.0 * static_cast<double>(j) / widths[ax]);
-        }
+    tab.pairs_t = l.cfg.d_t / 2;
+    tab.pairs_th = (l.cfg.d_t + l.cfg.d_h) / 2;
     RopeArgs a{static_cast<const __nv_bfloat16 *>(l.x), static_cast<__nv_bfloat16 *>(l.y), l.pos, l.n_valid,
                l.n_heads, l.out_scale, l.xb, l.xt, l.xh, l.yb, l.yt, l.yh, l.pb};
     dim3 grid(l.n_tokens, l.n_batch);
@@ -262,10 +308,17 @@ int pool_launch(const PoolLaunch &l) {
     a.frame_t = l.frame_t;
     a.pos_out = l.pos_out;
     a.pos_b = l.pos_b;
-    a.total = static_cast<int64_t>(l.n_batch) * l.n_frames * a.cells * l.n_heads * (D / 8);
+    a.total = static_cast<int64_t>(a.cells) * l.n_heads * (D / 8);   // threads per frame
+    if (a.total > 0x7fffffff || l.n_frames > 65535 || l.n_batch > 65535)
+        return set_error(SR_ERR_INVALID_ARG, "history_compress: too many cells, frames or sessions");
     if (a.total > 0) {
-        const int64_t blocks = (a.total + 255) / 256;
-        pool_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, l.stream>>>(a);
+        const dim3 blocks(static_cast<unsigned>((a.total + 255) / 256), l.n_frames, l.n_batch);
+        if (a.pool_h == 2 && a.pool_w == 2)
+            pool_kernel<D, 2, 2><<<blocks, 256, 0, l.stream>>>(a);
+        else if (a.pool_h == 4 && a.pool_w == 4)
+            pool_kernel<D, 4, 4><<<blocks, 256, 0, l.stream>>>(a);
+        else
+            pool_kernel<D, 0, 0><<<blocks, 256, 0, l.stream>>>(a);
     }
     if (l.slot_of_src) {
         const int64_t n = static_cast<int64_t>(l.n_frames) * l.cfg.grid_h * l.cfg.grid_w;
@@ -293,9 +346,11 @@ int append_launch(const AppendLaunch &l) {
     a.buf_tokens = l.buf_tokens;
     a.dst_token = l.dst_token;
     a.sb = l.sb; a.st = l.st; a.sh = l.sh; a.psb = l.psb;
-    a.total = static_cast<int64_t>(l.n_batch) * l.n_tokens * l.n_heads * (D / 8);
-    const int64_t blocks = (a.total + 255) / 256;
-    append_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, l.stream>>>(a);
+    a.total = static_cast<int64_t>(l.n_tokens) * l.n_heads * (D / 8);   // threads per session
+    if (a.total > 0x7fffffff || l.n_batch > 65535)
+        return set_error(SR_ERR_INVALID_ARG, "kv_append: too many tokens or sessions");
+    const dim3 blocks(static_cast<unsigned>((a.total + 255) / 256), l.n_batch);
+    append_kernel<D><<<blocks, 256, 0, l.stream>>>(a);
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? SR_OK : set_cuda_error("kv_append launch", e);
 }

@@ -234,17 +234,15 @@ class StreamingWindow:
                           stream=stream)
 
     def rotate(self, q: torch.Tensor, stream=None) -> None:
-        """a3: RoPE of the chunk queries into q_att and of every non-prompt
-        window segment from k_raw into k_att, with the current template."""
+        """a3: RoPE of the chunk queries into q_att, and of every non-prompt
+        window slot from k_raw into k_att with the current template.  The
+        window part is one launch over the contiguous slots after the prompt;
+        padded slots hold zeros (position 0) and stay zeros."""
         capi.sr_rope3d_apply(q, self.q_att.permute(0, 2, 1, 3), self.q_pos, self.split, self.base,
                              n_valid=self.q_len, stream=stream)
-        for si, name in enumerate(self.segments):
-            if name == "prompt":
-                continue
-            off, cap = self.seg[name]
-            capi.sr_rope3d_apply(self.seg_view(self.k_raw, name), self.seg_view(self.k_att, name),
-                                 self.pos[:, off:off + cap], self.split, self.base,
-                                 n_valid=self.seg_valid[si], stream=stream)
+        off = self.seg["prompt"][1]
+        capi.sr_rope3d_apply(self.k_raw[:, :, off:].permute(0, 2, 1, 3), self.k_att[:, :, off:].permute(0, 2, 1, 3),
+                             self.pos[:, off:], self.split, self.base, stream=stream)
 
     def attend(self, stream=None) -> torch.Tensor:
         """a4: fused chunk attention -> o [B, q_cap, H, D] (and lse)."""
