@@ -52,6 +52,7 @@ def _load():
                                      ctypes.c_int, ctypes.c_int, ctypes.c_long]
             lib.sro_attention.argtypes = [dp, dp, dp, lp, ctypes.c_long, ctypes.c_long, ctypes.c_int,
                                           ctypes.c_double, dp, dp]
+            lib.sro_rms_norm.argtypes = [dp, dp, dp, ctypes.c_long, ctypes.c_int, ctypes.c_double]
             lib.sro_num_threads.restype = ctypes.c_int
             lib.sro_set_num_threads.argtypes = [ctypes.c_int]
             _lib = lib
@@ -90,6 +91,18 @@ def rope3d(x, pos, split: Tuple[int, int, int], base: float = 10000.0) -> np.nda
     pf = np.ascontiguousarray(np.repeat(pos.reshape(n, 3), per, axis=0))
     y = np.empty_like(xf)
     _load().sro_rope3d(_dp(xf), _dp(y), _dp(pf), xf.shape[0], D, split[0], split[1], split[2], float(base))
+    return y.reshape(x.shape)
+
+
+def rms_norm(x, gamma, eps: float) -> np.ndarray:
+    """Per-vector RMSNorm over the last axis with gain gamma [D]."""
+    x = _f64(x)
+    g = _f64(gamma).reshape(-1)
+    D = x.shape[-1]
+    assert g.size == D
+    xf = np.ascontiguousarray(x.reshape(-1, D))
+    y = np.empty_like(xf)
+    _load().sro_rms_norm(_dp(xf), _dp(y), _dp(g), xf.shape[0], D, float(eps))
     return y.reshape(x.shape)
 
 

@@ -62,6 +62,30 @@ void sro_rope3d(const double *x, double *y, const double *pos, long n, int D,
 }
 
 /*
+ * QK normalisation: RMSNorm of every head vector before RoPE.
+ *
+ * Source: "MiniMax-H3 deep dive" (fiv.co.kr), tensor-name paragraph: the
+ * attention carries norm_q / norm_k (QK normalisation) next to to_q / to_k.
+ * Reading: per head vector of length D, with a learned gain g[D]:
+ *     y[d] = x[d] / sqrt(mean_d(x[d]^2) + eps) * g[d]
+ *
+ * x, y: [n][D]; g: [D].
+ */
+void sro_rms_norm(const double *x, double *y, const double *g, long n, int D, double eps)
+{
+    long i;
+#pragma omp parallel for schedule(static)
+    for (i = 0; i < n; ++i) {
+        const double *xi = x + i * (long)D;
+        double *yi = y + i * (long)D;
+        double ss = 0.0;
+        for (int d = 0; d < D; ++d) ss += xi[d] * xi[d];
+        const double inv = 1.0 / sqrt(ss / (double)D + eps);
+        for (int d = 0; d < D; ++d) yi[d] = xi[d] * inv * g[d];
+    }
+}
+
+/*
  * Spatial average pooling of one history tier.
  *
  * Source: "AlayaRenderer-Flash" (aitrends.kr), key contributions and
