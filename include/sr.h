@@ -91,6 +91,32 @@ int sr_rope3d_apply(const void *x, void *y, const float *pos,
                     int64_t y_batch_stride, int64_t y_token_stride, int64_t y_head_stride,
                     int64_t pos_batch_stride, void *stream);
 
+/* QK normalisation fused with the 3-D RoPE and the cache write.
+ *
+ * Defined by: "MiniMax-H3 deep dive" (fiv.co.kr), tensor-name paragraph
+ * (norm_q / norm_k beside to_q / to_k: QK normalisation in the shared
+ * attention); "StreamRender-H3" (molayo1419.me), causal VAE section (qk-norm,
+ * RoPE and KV-cache write fused in one kernel).
+ *
+ * Reading: per head vector (length D), RMSNorm with a learned gain, then the
+ * rotation of sr_rope3d_apply:
+ *   u = x / sqrt(mean_d(x[d]^2) + eps) * gamma      (fp32)
+ *   y = out_scale * R(pos) u                         (bf16 RNE)
+ *   y_raw = u                                        (bf16 RNE, optional)
+ * Arguments as in sr_rope3d_apply, plus gamma: fp32 [head_dim] on the device
+ * (16-byte aligned); eps >= 0; y_raw: optional output with its own strides
+ * (element (b, n, h, d) at y_raw + b*yraw_batch_stride + n*yraw_token_stride
+ * + h*yraw_head_stride + d), NULL = not written.
+ * Requires n_heads <= 64 at head_dim 128 (<= 128 at head_dim 64).
+ */
+int sr_qknorm_rope3d_apply(const void *x, void *y, void *y_raw, const float *gamma, float eps,
+                           const float *pos, int32_t n_batch, int32_t n_tokens, int32_t n_heads,
+                           int32_t head_dim, const int32_t *n_valid_dev, sr_rope_cfg cfg, float out_scale,
+                           int64_t x_batch_stride, int64_t x_token_stride, int64_t x_head_stride,
+                           int64_t y_batch_stride, int64_t y_token_stride, int64_t y_head_stride,
+                           int64_t yraw_batch_stride, int64_t yraw_token_stride, int64_t yraw_head_stride,
+                           int64_t pos_batch_stride, void *stream);
+
 /* ------------------------------------------------------------------------ */
 /* History-tier pooling.
  *
@@ -159,6 +185,32 @@ int sr_kv_append(void *k_buf, void *v_buf, float *pos_buf,
                  int32_t n_tokens, const int32_t *n_valid_dev,
                  int64_t src_batch_stride, int64_t src_token_stride, int64_t src_head_stride,
                  int64_t pos_src_batch_stride, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Index gather / scatter of token rows (window partition and merge).
+ *
+ * Defined by: "StreamRender-H3" (molayo1419.me), causal VAE section: the
+ * decoder's attention uses non-overlapping 16x16 token windows, shifted by
+ * half a window every other layer, with each window's KV in a preallocated
+ * ring buffer; window partition and merge are done by index gathers.
+ *
+ * Gather:  dst[b][s][h][:] = idx[b][s] >= 0 ? src[idx[b][s]][h][:] : 0
+ *   src element (t, h, d) at src + t*src_token_stride + h*src_head_stride + d
+ *   dst element (b, s, h, d) at dst + b*dst_batch_stride + s*dst_slot_stride + h*dst_head_stride + d
+ *   src_pos / dst_pos (optional, together): fp32 (t, h, w) triples, src_pos
+ *   [tokens][3], dst_pos[b][s] at dst_pos + b*dst_pos_batch_stride + 3*s
+ *   (zero for idx < 0).
+ * Scatter: dst[idx[b][s]][h][:] = src[b][s][h][:] for every idx[b][s] >= 0
+ *   (the slotted layout is the source; indices must not repeat).
+ * idx: int32 [n_batch][n_slots] on the device.  head_dim in {64, 128}.
+ */
+int sr_gather_tokens(void *dst, const void *src, const int32_t *idx, int32_t n_batch, int32_t n_slots,
+                     int32_t n_heads, int32_t head_dim, int64_t src_token_stride, int64_t src_head_stride,
+                     int64_t dst_batch_stride, int64_t dst_slot_stride, int64_t dst_head_stride,
+                     const float *src_pos, float *dst_pos, int64_t dst_pos_batch_stride, void *stream);
+int sr_scatter_tokens(void *dst, const void *src, const int32_t *idx, int32_t n_batch, int32_t n_slots,
+                      int32_t n_heads, int32_t head_dim, int64_t dst_token_stride, int64_t dst_head_stride,
+                      int64_t src_batch_stride, int64_t src_slot_stride, int64_t src_head_stride, void *stream);
 
 /* ------------------------------------------------------------------------ */
 /* Fused chunk attention over [prompt | context | chunk] KV segments.

@@ -18,7 +18,7 @@ from typing import Dict, List, Optional, Sequence
 
 import numpy as np
 
-from . import attention, layout, pool, rope3d, _f64
+from . import attention, layout, pool, rms_norm, rope3d, _f64
 
 
 def pooled_tier(spec, frames_k, frames_v, ph: int, pw: int):
@@ -77,17 +77,26 @@ def session_kv(spec, inp, heads: Optional[Sequence[int]] = None) -> List[Dict]:
 
 
 def session_reference(spec, inp, heads: Optional[Sequence[int]] = None,
-                      rows: Optional[Sequence[int]] = None):
+                      rows: Optional[Sequence[int]] = None, qk_norm=None):
     """O [n_rows, n_heads_sel, D] and LSE [n_rows, n_heads_sel] in fp64 for the
-    chunk queries ``rows`` (default all) and ``heads`` (default all)."""
+    chunk queries ``rows`` (default all) and ``heads`` (default all).
+
+    qk_norm: optional (gamma_q, gamma_k, eps).  Reading of the norm_q /
+    norm_k tensors ("MiniMax-H3 deep dive", tensor-name paragraph): every
+    query and key vector (pooled keys after pooling) is RMS-normalised with
+    its gain before RoPE."""
     H, D = spec.n_heads, spec.head_dim
     heads = list(range(H)) if heads is None else list(heads)
     segs = session_kv(spec, inp, heads)
     k_all = np.concatenate([s["k"] for s in segs])
     v_all = np.concatenate([s["v"] for s in segs])
     p_all = np.concatenate([s["pos"] for s in segs])
+    if qk_norm is not None:
+        k_all = rms_norm(k_all, qk_norm[1], qk_norm[2])
     k_rot = rope3d(k_all, p_all, spec.rope_split, spec.rope_base)
     q = _f64(inp.q)[:, heads]
+    if qk_norm is not None:
+        q = rms_norm(q, qk_norm[0], qk_norm[2])
     q_pos = np.asarray(layout.chunk_positions(spec), dtype=np.float64)
     if rows is not None:
         rows = list(rows)
@@ -102,4 +111,68 @@ def session_reference(spec, inp, heads: Optional[Sequence[int]] = None,
         o[:, hi], lse[:, hi] = attention(np.ascontiguousarray(q_rot[:, hi]),
                                          np.ascontiguousarray(k_rot[:, hi]),
                                          np.ascontiguousarray(v_all[:, hi]), scale)
+    return o, lse
+
+
+def prefix_reference(spec, inp, mov, heads: Optional[Sequence[int]] = None, rows: Optional[Sequence[int]] = None):
+    """Attention of the fixed prefix's own queries (prompt then sink tokens)
+    over the prefix keys only.
+
+    Source: "StreamRender-H3" (molayo1419.me), streaming context section: the
+    prefix cache (text and image conditions, reference image, sink) is
+    computed once per denoising step; the fixed prefix attends only to
+    itself, the moving part to the whole window.  Reading: prefix = prompt +
+    sink segments; prompt queries unrotated like their keys, sink queries at
+    the sink frame's positions."""
+    H, D = spec.n_heads, spec.head_dim
+    heads = list(range(H)) if heads is None else list(heads)
+    segs = {s["name"]: s for s in session_kv(spec, inp, heads)}
+    names = [n for n in ("prompt", "sink") if n in segs]
+    k = np.concatenate([segs[n]["k"] for n in names])
+    v = np.concatenate([segs[n]["v"] for n in names])
+    pos = np.concatenate([segs[n]["pos"] for n in names])
+    k_rot = rope3d(k, pos, spec.rope_split, spec.rope_base)
+    q = _f64(mov.prefix_q)[:, heads]
+    q_pos = pos
+    if rows is not None:
+        q, q_pos = q[list(rows)], q_pos[list(rows)]
+    q_rot = rope3d(q, q_pos, spec.rope_split, spec.rope_base)
+    scale = 1.0 / np.sqrt(D)
+    o = np.empty((q_rot.shape[0], len(heads), D))
+    lse = np.empty((q_rot.shape[0], len(heads)))
+    for hi in range(len(heads)):
+        o[:, hi], lse[:, hi] = attention(np.ascontiguousarray(q_rot[:, hi]), np.ascontiguousarray(k_rot[:, hi]),
+                                         np.ascontiguousarray(v[:, hi]), scale)
+    return o, lse
+
+
+def moving_reference(spec, inp, mov, heads: Optional[Sequence[int]] = None, rows: Optional[Sequence[int]] = None):
+    """Attention of the moving part's queries (recent frames, then the chunk)
+    over the whole window, where the recent frames' keys and values are the
+    recomputed ones (only the recent history and the current chunk are
+    recomputed at inference; same source as prefix_reference)."""
+    H, D = spec.n_heads, spec.head_dim
+    heads = list(range(H)) if heads is None else list(heads)
+    segs = session_kv(spec, inp, heads)
+    for sg in segs:
+        if sg["name"] == "recent":
+            assert sg["k"].shape[0] == mov.recent_k.shape[0]
+            sg["k"] = _f64(mov.recent_k)[:, heads]
+            sg["v"] = _f64(mov.recent_v)[:, heads]
+            recent_pos = sg["pos"]
+    k = np.concatenate([sg["k"] for sg in segs])
+    v = np.concatenate([sg["v"] for sg in segs])
+    pos = np.concatenate([sg["pos"] for sg in segs])
+    k_rot = rope3d(k, pos, spec.rope_split, spec.rope_base)
+    q = np.concatenate([_f64(mov.recent_q)[:, heads], _f64(inp.q)[:, heads]])
+    q_pos = np.concatenate([recent_pos, np.asarray(layout.chunk_positions(spec), dtype=np.float64)])
+    if rows is not None:
+        q, q_pos = q[list(rows)], q_pos[list(rows)]
+    q_rot = rope3d(q, q_pos, spec.rope_split, spec.rope_base)
+    scale = 1.0 / np.sqrt(D)
+    o = np.empty((q_rot.shape[0], len(heads), D))
+    lse = np.empty((q_rot.shape[0], len(heads)))
+    for hi in range(len(heads)):
+        o[:, hi], lse[:, hi] = attention(np.ascontiguousarray(q_rot[:, hi]), np.ascontiguousarray(k_rot[:, hi]),
+                                         np.ascontiguousarray(v[:, hi]), scale)
     return o, lse

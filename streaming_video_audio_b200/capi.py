@@ -55,6 +55,11 @@ _SIGS = {
     "sr_get_last_error": ([], ctypes.c_char_p),
     "sr_rope3d_apply": ([_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, sr_rope_cfg, _f32,
                          _i64, _i64, _i64, _i64, _i64, _i64, _i64, _vp], ctypes.c_int),
+    "sr_qknorm_rope3d_apply": ([_vp, _vp, _vp, _vp, _f32, _vp, _i32, _i32, _i32, _i32, _vp, sr_rope_cfg, _f32,
+                                _i64, _i64, _i64, _i64, _i64, _i64, _i64, _i64, _i64, _i64, _vp], ctypes.c_int),
+    "sr_gather_tokens": ([_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i64, _i64, _i64, _i64, _i64, _vp, _vp, _i64, _vp],
+                         ctypes.c_int),
+    "sr_scatter_tokens": ([_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i64, _i64, _i64, _i64, _i64, _vp], ctypes.c_int),
     "sr_history_compress": ([_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, sr_pool_cfg,
                              _i64, _i64, _i64, _i64, _i64, _i64, _i64, _i64, _vp, _vp, _i64, _vp, _vp],
                             ctypes.c_int),
@@ -139,6 +144,79 @@ def sr_rope3d_apply(x: torch.Tensor, y: torch.Tensor, pos: Optional[torch.Tensor
     _check("sr_rope3d_apply", load().sr_rope3d_apply(
         _ptr(x), _ptr(y), _ptr(pos), B, N, H, D, _ptr(n_valid), cfg, float(out_scale),
         x.stride(0), x.stride(1), x.stride(2), y.stride(0), y.stride(1), y.stride(2), pb, _stream(stream)))
+
+
+def sr_qknorm_rope3d_apply(x: torch.Tensor, y: torch.Tensor, gamma: torch.Tensor, eps: float,
+                           pos: Optional[torch.Tensor], split: Sequence[int], base: float = 10000.0,
+                           out_scale: float = 1.0, n_valid: Optional[torch.Tensor] = None,
+                           y_raw: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Per-head RMSNorm (gain gamma: fp32 [D], contiguous) then RoPE.  x, y,
+    y_raw: [B, N, H, D] bf16 views (D contiguous); pos as in sr_rope3d_apply."""
+    _cuda(x, torch.bfloat16, "x")
+    _cuda(y, torch.bfloat16, "y")
+    _cuda(y_raw, torch.bfloat16, "y_raw")
+    _cuda(gamma, torch.float32, "gamma")
+    _cuda(pos, torch.float32, "pos")
+    _cuda(n_valid, torch.int32, "n_valid")
+    B, N, H, D = x.shape
+    if tuple(y.shape) != (B, N, H, D) or x.stride(3) != 1 or y.stride(3) != 1:
+        raise ValueError("x and y must be [B, N, H, D] with contiguous D")
+    if y_raw is not None and (tuple(y_raw.shape) != (B, N, H, D) or y_raw.stride(3) != 1):
+        raise ValueError("y_raw must be [B, N, H, D] with contiguous D")
+    if gamma.numel() != D or not gamma.is_contiguous():
+        raise ValueError("gamma must be contiguous fp32 [D]")
+    pb = 0
+    if pos is not None:
+        if tuple(pos.shape) != (B, N, 3) or pos.stride(1) != 3 or pos.stride(2) != 1:
+            raise ValueError("pos must be [B, N, 3] with token stride 3")
+        pb = pos.stride(0)
+    rs = y_raw.stride() if y_raw is not None else (0, 0, 0)
+    cfg = sr_rope_cfg(float(base), int(split[0]), int(split[1]), int(split[2]))
+    _check("sr_qknorm_rope3d_apply", load().sr_qknorm_rope3d_apply(
+        _ptr(x), _ptr(y), _ptr(y_raw), _ptr(gamma), float(eps), _ptr(pos), B, N, H, D, _ptr(n_valid), cfg,
+        float(out_scale), x.stride(0), x.stride(1), x.stride(2), y.stride(0), y.stride(1), y.stride(2),
+        rs[0], rs[1], rs[2], pb, _stream(stream)))
+
+
+def sr_gather_tokens(dst: torch.Tensor, src: torch.Tensor, idx: torch.Tensor, src_pos: Optional[torch.Tensor] = None,
+                     dst_pos: Optional[torch.Tensor] = None, stream=None) -> None:
+    """dst [B, S, H, D] view (D contiguous) <- rows of src [T, H, D] (view, D
+    contiguous) picked by idx int32 [B, S] (contiguous; < 0 -> zeros);
+    optional positions src_pos [T, 3] -> dst_pos [B, S, 3] (token stride 3)."""
+    for t, n in ((dst, "dst"), (src, "src")):
+        _cuda(t, torch.bfloat16, n)
+    _cuda(idx, torch.int32, "idx")
+    B, S, H, D = dst.shape
+    if src.dim() != 3 or src.shape[1:] != (H, D) or src.stride(2) != 1 or dst.stride(3) != 1:
+        raise ValueError("src must be [T, H, D] and dst [B, S, H, D] with contiguous D")
+    if tuple(idx.shape) != (B, S) or not idx.is_contiguous():
+        raise ValueError("idx must be contiguous int32 [B, S]")
+    pb = 0
+    if dst_pos is not None:
+        _cuda(dst_pos, torch.float32, "dst_pos")
+        _cuda(src_pos, torch.float32, "src_pos")
+        if tuple(dst_pos.shape) != (B, S, 3) or dst_pos.stride(1) != 3 or not src_pos.is_contiguous():
+            raise ValueError("dst_pos must be [B, S, 3] (token stride 3), src_pos contiguous [T, 3]")
+        pb = dst_pos.stride(0)
+    _check("sr_gather_tokens", load().sr_gather_tokens(
+        _ptr(dst), _ptr(src), _ptr(idx), B, S, H, D, src.stride(0), src.stride(1), dst.stride(0), dst.stride(1),
+        dst.stride(2), _ptr(src_pos), _ptr(dst_pos), pb, _stream(stream)))
+
+
+def sr_scatter_tokens(dst: torch.Tensor, src: torch.Tensor, idx: torch.Tensor, stream=None) -> None:
+    """Rows of src [B, S, H, D] (view, D contiguous) to dst [T, H, D] at
+    idx [B, S] (int32, contiguous; < 0 skipped; indices must not repeat)."""
+    for t, n in ((dst, "dst"), (src, "src")):
+        _cuda(t, torch.bfloat16, n)
+    _cuda(idx, torch.int32, "idx")
+    B, S, H, D = src.shape
+    if dst.dim() != 3 or dst.shape[1:] != (H, D) or dst.stride(2) != 1 or src.stride(3) != 1:
+        raise ValueError("dst must be [T, H, D] and src [B, S, H, D] with contiguous D")
+    if tuple(idx.shape) != (B, S) or not idx.is_contiguous():
+        raise ValueError("idx must be contiguous int32 [B, S]")
+    _check("sr_scatter_tokens", load().sr_scatter_tokens(
+        _ptr(dst), _ptr(src), _ptr(idx), B, S, H, D, dst.stride(0), dst.stride(1), src.stride(0), src.stride(1),
+        src.stride(2), _stream(stream)))
 
 
 def sr_history_compress(k_in: Optional[torch.Tensor], v_in: Optional[torch.Tensor],

@@ -98,6 +98,116 @@ int sr_rope3d_apply(const void *x, void *y, const float *pos, int32_t n_batch, i
     return launch_rope3d(l);
 }
 
+int sr_qknorm_rope3d_apply(const void *x, void *y, void *y_raw, const float *gamma, float eps, const float *pos,
+                           int32_t n_batch, int32_t n_tokens, int32_t n_heads, int32_t head_dim,
+                           const int32_t *n_valid_dev, sr_rope_cfg cfg, float out_scale, int64_t x_batch_stride,
+                           int64_t x_token_stride, int64_t x_head_stride, int64_t y_batch_stride,
+                           int64_t y_token_stride, int64_t y_head_stride, int64_t yraw_batch_stride,
+                           int64_t yraw_token_stride, int64_t yraw_head_stride, int64_t pos_batch_stride,
+                           void *stream) {
+    g_last_error[0] = 0;
+    if (!gamma) return set_error(SR_ERR_INVALID_ARG, "qknorm_rope3d: gamma is NULL");
+    if (reinterpret_cast<uintptr_t>(gamma) & 15u)
+        return set_error(SR_ERR_INVALID_ARG, "qknorm_rope3d: gamma must be 16-byte aligned");
+    if (!(eps >= 0.f)) return set_error(SR_ERR_INVALID_ARG, "qknorm_rope3d: eps must be >= 0");
+    if ((head_dim == 64 || head_dim == 128) && n_heads > rope_norm_max_heads(head_dim))
+        return set_error(SR_ERR_UNSUPPORTED, "qknorm_rope3d: at most %d heads of %d", rope_norm_max_heads(head_dim),
+                         head_dim);
+    if (y_raw && (!aligned16(y_raw) || !stride_ok(yraw_batch_stride) || !stride_ok(yraw_token_stride) ||
+                  !stride_ok(yraw_head_stride)))
+        return set_error(SR_ERR_INVALID_ARG, "qknorm_rope3d: y_raw must be 16-byte aligned with strides of 8");
+    // the rest of the validation is that of sr_rope3d_apply
+    if (n_batch < 0 || n_tokens < 0 || n_heads < 1 || n_batch > 65535)
+        return set_error(SR_ERR_INVALID_ARG, "qknorm_rope3d: bad sizes (batch %d, tokens %d, heads %d)", n_batch,
+                         n_tokens, n_heads);
+    if (head_dim != 64 && head_dim != 128)
+        return set_error(SR_ERR_UNSUPPORTED, "qknorm_rope3d: head_dim must be 64 or 128");
+    if (cfg.d_t < 0 || cfg.d_h < 0 || cfg.d_w < 0 || cfg.d_t % 8 || cfg.d_h % 8 || cfg.d_w % 8 ||
+        cfg.d_t + cfg.d_h + cfg.d_w != head_dim)
+        return set_error(SR_ERR_INVALID_ARG, "qknorm_rope3d: sub-blocks %d/%d/%d must be multiples of 8 summing to %d",
+                         cfg.d_t, cfg.d_h, cfg.d_w, head_dim);
+    if (!(cfg.base > 0.f)) return set_error(SR_ERR_INVALID_ARG, "qknorm_rope3d: base must be positive");
+    if (n_batch == 0 || n_tokens == 0) return SR_OK;
+    if (!x || !y) return set_error(SR_ERR_INVALID_ARG, "qknorm_rope3d: null tensor");
+    if (!aligned16(x) || !aligned16(y))
+        return set_error(SR_ERR_INVALID_ARG, "qknorm_rope3d: x and y must be 16-byte aligned");
+    if (!stride_ok(x_batch_stride) || !stride_ok(x_token_stride) || !stride_ok(x_head_stride) ||
+        !stride_ok(y_batch_stride) || !stride_ok(y_token_stride) || !stride_ok(y_head_stride))
+        return set_error(SR_ERR_INVALID_ARG, "qknorm_rope3d: strides must be multiples of 8 elements");
+    if (pos && (reinterpret_cast<uintptr_t>(pos) & 3u))
+        return set_error(SR_ERR_INVALID_ARG, "qknorm_rope3d: pos must be 4-byte aligned");
+    RopeLaunch l{x, y, pos, n_valid_dev, n_batch, n_tokens, n_heads, head_dim, cfg, out_scale,
+                 x_batch_stride, x_token_stride, x_head_stride, y_batch_stride, y_token_stride, y_head_stride,
+                 pos_batch_stride, static_cast<cudaStream_t>(stream)};
+    l.gamma = gamma;
+    l.eps = eps;
+    l.y_raw = y_raw;
+    l.rb = yraw_batch_stride;
+    l.rt = yraw_token_stride;
+    l.rh = yraw_head_stride;
+    return launch_rope3d(l);
+}
+
+static int gather_common(const char *name, void *dst, const void *src, const int32_t *idx, int32_t n_batch,
+                         int32_t n_slots, int32_t n_heads, int32_t head_dim, int64_t tok_t, int64_t tok_h,
+                         int64_t slot_b, int64_t slot_s, int64_t slot_h, GatherLaunch &l) {
+    if (n_batch < 0 || n_slots < 0 || n_heads < 1 || n_batch > 65535)
+        return set_error(SR_ERR_INVALID_ARG, "%s: bad sizes", name);
+    if (head_dim != 64 && head_dim != 128) return set_error(SR_ERR_UNSUPPORTED, "%s: head_dim must be 64 or 128", name);
+    if (n_batch == 0 || n_slots == 0) return -1;   // nothing to do
+    if (!dst || !src || !idx) return set_error(SR_ERR_INVALID_ARG, "%s: null pointer", name);
+    if (!aligned16(dst) || !aligned16(src)) return set_error(SR_ERR_INVALID_ARG, "%s: tensors must be 16-byte aligned", name);
+    for (int64_t st : {tok_t, tok_h, slot_b, slot_s, slot_h})
+        if (!stride_ok(st)) return set_error(SR_ERR_INVALID_ARG, "%s: strides must be multiples of 8", name);
+    l.idx = idx;
+    l.n_batch = n_batch;
+    l.n_slots = n_slots;
+    l.n_heads = n_heads;
+    l.head_dim = head_dim;
+    l.src_t = tok_t;
+    l.src_h = tok_h;
+    l.dst_b = slot_b;
+    l.dst_s = slot_s;
+    l.dst_h = slot_h;
+    return SR_OK;
+}
+
+int sr_gather_tokens(void *dst, const void *src, const int32_t *idx, int32_t n_batch, int32_t n_slots,
+                     int32_t n_heads, int32_t head_dim, int64_t src_token_stride, int64_t src_head_stride,
+                     int64_t dst_batch_stride, int64_t dst_slot_stride, int64_t dst_head_stride,
+                     const float *src_pos, float *dst_pos, int64_t dst_pos_batch_stride, void *stream) {
+    g_last_error[0] = 0;
+    GatherLaunch l{};
+    int rc = gather_common("gather_tokens", dst, src, idx, n_batch, n_slots, n_heads, head_dim, src_token_stride,
+                           src_head_stride, dst_batch_stride, dst_slot_stride, dst_head_stride, l);
+    if (rc != SR_OK) return rc < 0 ? SR_OK : rc;
+    if ((src_pos == nullptr) != (dst_pos == nullptr))
+        return set_error(SR_ERR_INVALID_ARG, "gather_tokens: src_pos and dst_pos go together");
+    l.dst = dst;
+    l.src = src;
+    l.src_pos = src_pos;
+    l.dst_pos = dst_pos;
+    l.pos_b = dst_pos_batch_stride;
+    l.scatter = false;
+    l.stream = static_cast<cudaStream_t>(stream);
+    return launch_gather(l);
+}
+
+int sr_scatter_tokens(void *dst, const void *src, const int32_t *idx, int32_t n_batch, int32_t n_slots,
+                      int32_t n_heads, int32_t head_dim, int64_t dst_token_stride, int64_t dst_head_stride,
+                      int64_t src_batch_stride, int64_t src_slot_stride, int64_t src_head_stride, void *stream) {
+    g_last_error[0] = 0;
+    GatherLaunch l{};
+    int rc = gather_common("scatter_tokens", dst, src, idx, n_batch, n_slots, n_heads, head_dim, dst_token_stride,
+                           dst_head_stride, src_batch_stride, src_slot_stride, src_head_stride, l);
+    if (rc != SR_OK) return rc < 0 ? SR_OK : rc;
+    l.dst = dst;
+    l.src = src;
+    l.scatter = true;
+    l.stream = static_cast<cudaStream_t>(stream);
+    return launch_gather(l);
+}
+
 int sr_history_compress(const void *k_in, const void *v_in, void *k_out, void *v_out, int32_t n_batch,
                         int32_t n_frames, int32_t n_heads, int32_t head_dim, sr_pool_cfg cfg, int64_t in_batch_stride,
                         int64_t in_frame_stride, int64_t in_token_stride, int64_t in_head_stride,

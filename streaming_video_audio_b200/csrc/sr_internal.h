@@ -58,8 +58,26 @@ struct RopeLaunch {
     float out_scale;
     int64_t xb, xt, xh, yb, yt, yh, pb;
     cudaStream_t stream;
+    const float *gamma = nullptr;   // non-null: RMSNorm each head vector first
+    float eps = 0.f;
+    void *y_raw = nullptr;          // optional normalised, unrotated copy
+    int64_t rb = 0, rt = 0, rh = 0;
 };
 int launch_rope3d(const RopeLaunch &a);
+int rope_norm_max_heads(int head_dim);
+
+struct GatherLaunch {
+    void *dst;
+    const void *src;
+    const int32_t *idx;
+    const float *src_pos;
+    float *dst_pos;
+    int32_t n_batch, n_slots, n_heads, head_dim;
+    int64_t src_t, src_h, dst_b, dst_s, dst_h, pos_b;
+    bool scatter;
+    cudaStream_t stream;
+};
+int launch_gather(const GatherLaunch &l);
 
 struct PoolLaunch {
     const void *k_in, *v_in;

@@ -52,6 +52,12 @@ struct RopeArgs {
     int32_t n_heads;
     float out_scale;
     int64_t xb, xt, xh, yb, yt, yh, pb;
+    // QK normalisation (norm kernels only): per-head RMSNorm with gain
+    // gamma[D]; y_raw (optional) receives the normalised vector before RoPE
+    const float *__restrict__ gamma;
+    float eps;
+    __nv_bfloat16 *__restrict__ y_raw;
+    int64_t rb, rt, rh;
 };
 
 // One CTA per (token, batch).  Thread t handles the 16-byte chunk
@@ -62,7 +68,11 @@ struct RopeArgs {
 // p * theta is formed in double and reduced to [-pi, pi] in double, so its
 // error does not grow with the position's magnitude; the small remainder goes
 // through fp32 sincosf.  The rotation itself runs in fp32.
-template <int D>
+// kNorm: RMSNorm of each head vector first (QK normalisation): the D/8
+// threads holding one head row reduce its sum of squares with shuffles, then
+// scale by rsqrt(mean + eps) * gamma before rotating.  Needs n_heads <=
+// kIters * (128 / (D/8)) so every thread runs the same shuffles.
+template <int D, bool kNorm>
 __global__ void __launch_bounds__(128) rope3d_kernel(const RopeArgs a, const RopeTable tab) {
     constexpr int kChunks = D / 8;
     constexpr int kHeadsPerPass = 128 / kChunks;
@@ -77,7 +87,14 @@ __global__ void __launch_bounds__(128) rope3d_kernel(const RopeArgs a, const Rop
 #pragma unroll
     for (int i = 0; i < kIters; ++i) {
         const int h = hp + i * kHeadsPerPass;
-        if (h < a.n_heads) u[i] = __ldg(reinterpret_cast<const uint4 *>(xt + h * a.xh));
+        u[i] = h < a.n_heads ? __ldg(reinterpret_cast<const uint4 *>(xt + h * a.xh)) : make_uint4(0, 0, 0, 0);
+    }
+    float g[8];
+    if constexpr (kNorm) {
+        const float4 g0 = __ldg(reinterpret_cast<const float4 *>(a.gamma + c * 8));
+        const float4 g1 = __ldg(reinterpret_cast<const float4 *>(a.gamma + c * 8 + 4));
+        g[0] = g0.x; g[1] = g0.y; g[2] = g0.z; g[3] = g0.w;
+        g[4] = g1.x; g[5] = g1.y; g[6] = g1.z; g[7] = g1.w;
     }
     // theta per pair, staged once per CTA: indexing the parameter table with a
     // per-thread index would serialise the constant-cache reads
@@ -108,17 +125,31 @@ __global__ void __launch_bounds__(128) rope3d_kernel(const RopeArgs a, const Rop
 #pragma unroll
     for (int i = 0; i < kIters; ++i) {
         const int h = hp + i * kHeadsPerPass;
+        if (kNorm && i * kHeadsPerPass >= a.n_heads) break;   // uniform: no head of this pass exists
+        float f[8], r[8];
+        unpack8(u[i], f);
+        if constexpr (kNorm) {
+            float ss = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
+#pragma unroll
+            for (int off = kChunks / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+            const float inv = rsqrtf(ss * (1.0f / D) + a.eps);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] = f[e] * inv * g[e];
+            if (a.y_raw && h < a.n_heads)
+                *reinterpret_cast<uint4 *>(a.y_raw + b * a.rb + n * a.rt + h * a.rh + c * 8) = pack8(f);
+        }
         if (h < a.n_heads) {
-            float f[8], g[8];
-            unpack8(u[i], f);
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                g[2 * k] = f[2 * k] * cs[k] - f[2 * k + 1] * sn[k];
-                g[2 * k + 1] = f[2 * k] * sn[k] + f[2 * k + 1] * cs[k];
+                r[2 * k] = f[2 * k] * cs[k] - f[2 * k + 1] * sn[k];
+                r[2 * k + 1] = f[2 * k] * sn[k] + f[2 * k + 1] * cs[k];
             }
-            *reinterpret_cast<uint4 *>(yt + h * a.yh) = pack8(g);
+            *reinterpret_cast<uint4 *>(yt + h * a.yh) = pack8(r);
         }
     }
+    if constexpr (kNorm) return;   // the host guarantees n_heads fits the passes above
     for (int h = hp + kIters * kHeadsPerPass; h < a.n_heads; h += kHeadsPerPass) {   // very many heads
         float f[8], g[8];
         unpack8(__ldg(reinterpret_cast<const uint4 *>(xt + h * a.xh)), f);
@@ -270,7 +301,79 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendArgs a) {
     }
 }
 
+// ============================================================== index gather / scatter
+// Token rows move between a token list and a slotted layout (window-major
+// buffers, ring slots).  One thread per (batch, slot, head, 16-byte chunk).
+struct GatherArgs {
+    void *__restrict__ dst;
+    const void *__restrict__ src;
+    const int32_t *__restrict__ idx;   // [n_batch][n_slots]: source token, or < 0
+    const float *__restrict__ src_pos; // gather only: [tokens][3] or null
+    float *__restrict__ dst_pos;       // gather only: [n_batch][n_slots][3] or null
+    int32_t n_slots, n_heads;
+    int64_t src_t, src_h, dst_b, dst_s, dst_h, pos_b;
+    int64_t total;                     // threads per batch entry
+};
+
+// dst[b][s][h][:] = idx >= 0 ? src[idx][h][:] : 0   (and the positions likewise)
 template <int D>
+__global__ void __launch_bounds__(256) gather_kernel(const GatherArgs a) {
+    constexpr int kChunks = D / 8;
+    const uint32_t i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= static_cast<uint32_t>(a.total)) return;
+    const int b = blockIdx.y;
+    const int c = static_cast<int>(i % kChunks);
+    const uint32_t hs = i / kChunks;
+    const int h = static_cast<int>(hs % static_cast<uint32_t>(a.n_heads));
+    const int sl = static_cast<int>(hs / static_cast<uint32_t>(a.n_heads));
+    const int t = a.idx[static_cast<int64_t>(b) * a.n_slots + sl];
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (t >= 0)
+        v = __ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(a.src) + t * a.src_t +
+                                                   h * a.src_h + c * 8));
+    *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.dst) + b * a.dst_b + sl * a.dst_s + h * a.dst_h + c * 8) = v;
+    if (a.dst_pos && h == 0 && c == 0) {
+        float *pd = a.dst_pos + b * a.pos_b + 3 * static_cast<int64_t>(sl);
+        for (int e = 0; e < 3; ++e) pd[e] = t >= 0 ? a.src_pos[3 * static_cast<int64_t>(t) + e] : 0.f;
+    }
+}
+
+// dst[idx][h][:] = src[b][s][h][:] for idx >= 0 (dst/src roles of GatherArgs:
+// src is the slotted layout here, dst the token list)
+template <int D>
+__global__ void __launch_bounds__(256) scatter_kernel(const GatherArgs a) {
+    constexpr int kChunks = D / 8;
+    const uint32_t i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= static_cast<uint32_t>(a.total)) return;
+    const int b = blockIdx.y;
+    const int c = static_cast<int>(i % kChunks);
+    const uint32_t hs = i / kChunks;
+    const int h = static_cast<int>(hs % static_cast<uint32_t>(a.n_heads));
+    const int sl = static_cast<int>(hs / static_cast<uint32_t>(a.n_heads));
+    const int t = a.idx[static_cast<int64_t>(b) * a.n_slots + sl];
+    if (t < 0) return;
+    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(a.src) + b * a.dst_b +
+                                                          sl * a.dst_s + h * a.dst_h + c * 8));
+    *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.dst) + t * a.src_t + h * a.src_h + c * 8) = v;
+}
+
+template <int D>
+int gather_launch(const GatherLaunch &l) {
+    GatherArgs a{l.dst, l.src, l.idx, l.src_pos, l.dst_pos, l.n_slots, l.n_heads,
+                 l.src_t, l.src_h, l.dst_b, l.dst_s, l.dst_h, l.pos_b,
+                 static_cast<int64_t>(l.n_slots) * l.n_heads * (D / 8)};
+    if (a.total > 0x7fffffff || l.n_batch > 65535)
+        return set_error(SR_ERR_INVALID_ARG, "gather/scatter: too many slots or batch entries");
+    const dim3 grid(static_cast<unsigned>((a.total + 255) / 256), l.n_batch);
+    if (l.scatter)
+        scatter_kernel<D><<<grid, 256, 0, l.stream>>>(a);
+    else
+        gather_kernel<D><<<grid, 256, 0, l.stream>>>(a);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SR_OK : set_cuda_error("gather/scatter launch", e);
+}
+
+template <int D, bool kNorm>
 int rope_launch(const RopeLaunch &l) {
     RopeTable tab{};
     const int widths[3] = {l.cfg.d_t, l.cfg.d_h, l.cfg.d_w};
@@ -281,9 +384,10 @@ int rope_launch(const RopeLaunch &l) {
     tab.pairs_t = l.cfg.d_t / 2;
     tab.pairs_th = (l.cfg.d_t + l.cfg.d_h) / 2;
     RopeArgs a{static_cast<const __nv_bfloat16 *>(l.x), static_cast<__nv_bfloat16 *>(l.y), l.pos, l.n_valid,
-               l.n_heads, l.out_scale, l.xb, l.xt, l.xh, l.yb, l.yt, l.yh, l.pb};
+               l.n_heads, l.out_scale, l.xb, l.xt, l.xh, l.yb, l.yt, l.yh, l.pb,
+               l.gamma, l.eps, static_cast<__nv_bfloat16 *>(l.y_raw), l.rb, l.rt, l.rh};
     dim3 grid(l.n_tokens, l.n_batch);
-    rope3d_kernel<D><<<grid, 128, 0, l.stream>>>(a, tab);
+    rope3d_kernel<D, kNorm><<<grid, 128, 0, l.stream>>>(a, tab);
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? SR_OK : set_cuda_error("rope3d launch", e);
 }
@@ -357,7 +461,12 @@ int append_launch(const AppendLaunch &l) {
 
 }  // namespace
 
-int launch_rope3d(const RopeLaunch &l) { return l.head_dim == 128 ? rope_launch<128>(l) : rope_launch<64>(l); }
+int launch_rope3d(const RopeLaunch &l) {
+    if (l.gamma) return l.head_dim == 128 ? rope_launch<128, true>(l) : rope_launch<64, true>(l);
+    return l.head_dim == 128 ? rope_launch<128, false>(l) : rope_launch<64, false>(l);
+}
+int rope_norm_max_heads(int head_dim) { return 8 * (128 / (head_dim / 8)); }
+int launch_gather(const GatherLaunch &l) { return l.head_dim == 128 ? gather_launch<128>(l) : gather_launch<64>(l); }
 int launch_history_compress(const PoolLaunch &l) {
     return l.head_dim == 128 ? pool_launch<128>(l) : pool_launch<64>(l);
 }

@@ -1,0 +1,148 @@
+"""Shifted-window attention with ring-buffer KV, as in a causal streaming VAE
+decoder.
+
+Source: "StreamRender-H3" (molayo1419.me), causal VAE section:
+  * each call decodes 2 latent frames; every layer attends only to the KV of
+    the 2 current and the 4 previous latent frames, never to future frames;
+  * non-overlapping 16x16 token windows, shifted by half a window every
+    other layer to exchange information between neighbours;
+  * each window's KV lives in a preallocated ring buffer; position encoding
+    and the cache write happen once; window partition and merge are index
+    gathers; empty cache slots are hidden by per-slot valid lengths instead
+    of a mask.
+
+Readings: inside a call the two current frames see each other (causality at
+the granularity of a call); RoPE on (t, h, w) with t the absolute latent
+frame index, applied once when a frame enters the ring (attention only sees
+position differences); a window's tokens are packed valid-first (attention is
+invariant to key order), so partial windows at the grid edge are ragged
+segments.
+
+Everything runs in the library's kernels: sr_gather_tokens (partition),
+sr_rope3d_apply (positions, cache write), sr_chunk_attention_fwd (attention:
+batch = windows, segments = ring slots) and sr_scatter_tokens (merge).
+"""
+from __future__ import annotations
+
+import math
+from typing import List, Sequence
+
+import numpy as np
+import torch
+
+from . import capi
+
+
+class WindowPartition:
+    """Windows of `window` x `window` tokens tiling a gh x gw grid whose origin
+    is moved by -shift (shift = window / 2 on alternate layers)."""
+
+    def __init__(self, gh: int, gw: int, window: int = 16, shift: int = 0):
+        self.gh, self.gw, self.window, self.shift = gh, gw, window, shift
+        self.tokens: List[List[int]] = []   # row-major token indices of each window (valid only)
+        for r0 in range(-shift, gh, window):
+            for c0 in range(-shift, gw, window):
+                rows = range(max(r0, 0), min(r0 + window, gh))
+                cols = range(max(c0, 0), min(c0 + window, gw))
+                toks = [r * gw + c for r in rows for c in cols]
+                if toks:
+                    self.tokens.append(toks)
+        self.n_windows = len(self.tokens)
+        self.counts = np.array([len(t) for t in self.tokens], dtype=np.int32)
+
+    def frame_index(self, frames: int) -> np.ndarray:
+        """[n_windows][frames * window^2] int32: the windows' tokens of `frames`
+        consecutive frames packed valid-first (frame f's tokens offset by
+        f * gh * gw), padded with -1."""
+        slots = frames * self.window * self.window
+        out = np.full((self.n_windows, slots), -1, dtype=np.int32)
+        per = self.gh * self.gw
+        for w, toks in enumerate(self.tokens):
+            idx = [f * per + t for f in range(frames) for t in toks]
+            out[w, :len(idx)] = idx
+        return out
+
+
+class RingWindowAttention:
+    """One layer's windowed attention with a per-window KV ring of
+    (current + history) latent frames."""
+
+    def __init__(self, grid_hw, n_heads: int, head_dim: int, rope_split, shift: int = 0, window: int = 16,
+                 frames_per_call: int = 2, history_frames: int = 4, rope_base: float = 10000.0, device="cuda"):
+        self.part = WindowPartition(grid_hw[0], grid_hw[1], window, shift)
+        self.H, self.D = n_heads, head_dim
+        self.split, self.base = tuple(rope_split), rope_base
+        self.fpc, self.slots = frames_per_call, frames_per_call + history_frames
+        self.slot_cap = window * window
+        self.device = torch.device(device)
+        W, H, D, S = self.part.n_windows, n_heads, head_dim, self.slot_cap
+        kw = dict(device=self.device)
+        self.k_ring = torch.zeros(W, H, self.slots * S, D, dtype=torch.bfloat16, **kw)
+        self.v_ring = torch.zeros(W, H, self.slots * S, D, dtype=torch.bfloat16, **kw)
+        self.q_cap = self.fpc * S
+        self.q_tmp = torch.zeros(W, self.q_cap, H, D, dtype=torch.bfloat16, **kw)
+        self.k_tmp = torch.zeros(W, S, H, D, dtype=torch.bfloat16, **kw)
+        self.q_att = torch.zeros(W, H, self.q_cap, D, dtype=torch.bfloat16, **kw)
+        self.o_win = torch.zeros(W, self.q_cap, H, D, dtype=torch.bfloat16, **kw)
+        self.lse = torch.zeros(W, H, self.q_cap, dtype=torch.float32, **kw)
+        self.pos_q = torch.zeros(W, self.q_cap, 3, dtype=torch.float32, **kw)
+        self.pos_k = torch.zeros(W, S, 3, dtype=torch.float32, **kw)
+        self.status = torch.zeros(1, dtype=torch.int32, **kw)
+        self.idx_q = torch.from_numpy(self.part.frame_index(self.fpc)).to(self.device)
+        per = self.part.gh * self.part.gw
+        one = self.part.frame_index(1)
+        self.idx_kv = [torch.from_numpy(np.where(one >= 0, one + f * per, -1).astype(np.int32)).to(self.device)
+                       for f in range(self.fpc)]
+        self.q_len = torch.from_numpy(self.fpc * self.part.counts).to(self.device)
+        # valid length of every ring slot after call c: slots written so far hold a window's count
+        self.kv_len_phase = []
+        for c in range(self.slots // self.fpc):
+            lens = np.zeros((W, self.slots), dtype=np.int32)
+            lens[:, :min(self.slots, (c + 1) * self.fpc)] = self.part.counts[:, None]
+            self.kv_len_phase.append(torch.from_numpy(lens).to(self.device))
+        ws = capi.sr_chunk_attention_workspace_bytes(W, H, D, self.q_cap)
+        self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, **kw) if ws else None
+        self.calls = 0
+
+    def frame_positions(self, t0: int) -> torch.Tensor:
+        """(t, h, w) of the current frames' tokens, t absolute."""
+        gh, gw = self.part.gh, self.part.gw
+        r, c = np.divmod(np.arange(gh * gw), gw)
+        pos = [np.stack([np.full(gh * gw, t0 + f), r, c], axis=1) for f in range(self.fpc)]
+        return torch.from_numpy(np.concatenate(pos).astype(np.float32)).to(self.device)
+
+    def __call__(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, t0: int,
+                 out: torch.Tensor = None, stream=None) -> torch.Tensor:
+        """q, k, v: the current frames' tokens [frames_per_call * gh * gw, H, D]
+        (token-major, before RoPE); t0: absolute latent index of the first
+        current frame.  Returns o of the same shape."""
+        n_tok = self.fpc * self.part.gh * self.part.gw
+        assert q.shape == (n_tok, self.H, self.D) and k.shape == q.shape and v.shape == q.shape
+        if out is None:
+            out = torch.zeros_like(q)
+        W, H, D, S = self.part.n_windows, self.H, self.D, self.slot_cap
+        pos = self.frame_positions(t0)
+        slot0 = (self.calls * self.fpc) % self.slots
+        for f in range(self.fpc):
+            sl = (slot0 + f) % self.slots
+            ring_k = self.k_ring[:, :, sl * S:(sl + 1) * S]
+            ring_v = self.v_ring[:, :, sl * S:(sl + 1) * S]
+            # V straight into its ring slot; K through a staging buffer for its one-time RoPE
+            self._gather(ring_v.permute(0, 2, 1, 3), v, self.idx_kv[f], stream=stream)
+            self._gather(self.k_tmp, k, self.idx_kv[f], pos=pos, pos_out=self.pos_k, stream=stream)
+            capi.sr_rope3d_apply(self.k_tmp, ring_k.permute(0, 2, 1, 3), self.pos_k, self.split, self.base,
+                                 stream=stream)
+        self._gather(self.q_tmp, q, self.idx_q, pos=pos, pos_out=self.pos_q, stream=stream)
+        capi.sr_rope3d_apply(self.q_tmp, self.q_att.permute(0, 2, 1, 3), self.pos_q, self.split, self.base,
+                             stream=stream)
+        phase = min(self.calls, len(self.kv_len_phase) - 1)
+        capi.sr_chunk_attention_fwd(self.q_att, self.k_ring, self.v_ring, self.o_win, self.lse,
+                                    [S] * self.slots, self.kv_len_phase[phase], self.q_len, 1.0 / math.sqrt(D),
+                                    self.status, workspace=self.workspace, stream=stream)
+        capi.sr_scatter_tokens(out, self.o_win, self.idx_q, stream=stream)
+        self.calls += 1
+        return out
+
+    def _gather(self, dst, src, idx, pos=None, pos_out=None, stream=None):
+        """dst [W, slots, H, D] view <- src tokens [T, H, D] by idx [W, slots]."""
+        capi.sr_gather_tokens(dst, src, idx, src_pos=pos, dst_pos=pos_out, stream=stream)

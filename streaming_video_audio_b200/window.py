@@ -124,7 +124,12 @@ class StreamingWindow:
     place afterwards.
     """
 
-    def __init__(self, specs: Sequence, device="cuda"):
+    def __init__(self, specs: Sequence, device="cuda", qk_norm=None):
+        """qk_norm: optional (gamma_q, gamma_k, eps) -- per-head RMSNorm gains
+        (fp32 [head_dim]) applied to queries and keys before RoPE.  With it
+        the window keeps keys before normalisation (pooling then averages the
+        projected latents) and every rotation normalises first, fused in one
+        kernel."""
         self.plans = [SessionPlan(s) for s in specs]
         p0 = self.plans[0]
         self.B, self.H, self.D = len(self.plans), p0.H, p0.D
@@ -163,6 +168,11 @@ class StreamingWindow:
             qpos[b, :p.chunk_len] = p.chunk_positions()
         self.q_pos = torch.from_numpy(qpos).to(self.device)
         self.scale = 1.0 / math.sqrt(D)
+        self.qk_norm = None
+        if qk_norm is not None:
+            gq, gk, eps = qk_norm
+            self.qk_norm = (torch.as_tensor(gq, dtype=torch.float32).to(self.device).contiguous(),
+                            torch.as_tensor(gk, dtype=torch.float32).to(self.device).contiguous(), float(eps))
 
     # ---------------------------------------------------------------- views
     def seg_view(self, buf: torch.Tensor, name: str) -> torch.Tensor:
@@ -220,9 +230,8 @@ class StreamingWindow:
                     fill[role] += ntok
                     f += 1
         # the prompt is never re-positioned: rotate (identity) once
-        pv = self.seg_view(self.k_raw, "prompt")
-        capi.sr_rope3d_apply(pv, self.seg_view(self.k_att, "prompt"), None, self.split, self.base,
-                             n_valid=self.seg_valid[0], stream=stream)
+        self._rope(self.seg_view(self.k_raw, "prompt"), self.seg_view(self.k_att, "prompt"), None, key=True,
+                   n_valid=self.seg_valid[0], stream=stream)
         # chunk positions are the fixed template
         off = self.seg["chunk"][0]
         self.pos[:, off:off + self.q_cap].copy_(self.q_pos)
@@ -238,11 +247,22 @@ class StreamingWindow:
         window slot from k_raw into k_att with the current template.  The
         window part is one launch over the contiguous slots after the prompt;
         padded slots hold zeros (position 0) and stay zeros."""
-        capi.sr_rope3d_apply(q, self.q_att.permute(0, 2, 1, 3), self.q_pos, self.split, self.base,
-                             n_valid=self.q_len, stream=stream)
+        self._rope(q, self.q_att.permute(0, 2, 1, 3), self.q_pos, key=False, n_valid=self.q_len, stream=stream)
+        self.rotate_keys(stream)
+
+    def rotate_keys(self, stream=None) -> None:
+        """RoPE of every non-prompt window slot from k_raw into k_att (one launch)."""
         off = self.seg["prompt"][1]
-        capi.sr_rope3d_apply(self.k_raw[:, :, off:].permute(0, 2, 1, 3), self.k_att[:, :, off:].permute(0, 2, 1, 3),
-                             self.pos[:, off:], self.split, self.base, stream=stream)
+        self._rope(self.k_raw[:, :, off:].permute(0, 2, 1, 3), self.k_att[:, :, off:].permute(0, 2, 1, 3),
+                   self.pos[:, off:], key=True, stream=stream)
+
+    def _rope(self, x, y, pos, key: bool, n_valid=None, stream=None) -> None:
+        if self.qk_norm is None:
+            capi.sr_rope3d_apply(x, y, pos, self.split, self.base, n_valid=n_valid, stream=stream)
+        else:
+            gq, gk, eps = self.qk_norm
+            capi.sr_qknorm_rope3d_apply(x, y, gk if key else gq, eps, pos, self.split, self.base, n_valid=n_valid,
+                                        stream=stream)
 
     def attend(self, stream=None) -> torch.Tensor:
         """a4: fused chunk attention -> o [B, q_cap, H, D] (and lse)."""
@@ -271,6 +291,79 @@ class StreamingWindow:
         o = self.step(*staging, stream=stream)
         o_host.copy_(o, non_blocking=True)
         return o_host
+
+    # ---------------------------------------------------------------- prefix / moving part
+    # "StreamRender-H3" (molayo1419.me), streaming context section: the fixed
+    # prefix (conditions, reference, sink) is cached once per denoising step
+    # and attends only to itself; the moving part (recent history and the
+    # current chunk) is recomputed each step and attends to the whole window.
+    # A separate cache per denoising step ("bank") is a separate batch entry.
+    def prefix_positions(self) -> np.ndarray:
+        """[B, prefix_cap, 3] positions of the prefix queries: prompt (0) then sink tokens."""
+        lens = [p.lengths["prompt"] + p.lengths.get("sink", 0) for p in self.plans]
+        out = np.zeros((self.B, max(lens), 3), dtype=np.float32)
+        for b, p in enumerate(self.plans):
+            sink = [(t, n) for role, t, _, _, n in p.context if role == "sink"]
+            rows = [np.zeros((p.lengths["prompt"], 3), np.float32)] + [p.grid_positions(t, n) for t, n in sink]
+            x = np.concatenate(rows)
+            out[b, :x.shape[0]] = x
+        return out
+
+    def attend_prefix(self, q_prefix: torch.Tensor, stream=None) -> torch.Tensor:
+        """Prefix-self attention: queries of the prefix tokens (prompt, then
+        sink), token-major [B, prefix_cap, H, D] before RoPE, over the prefix
+        keys only.  Returns o [B, prefix_cap, H, D] (rows past a session's
+        prefix length are left alone)."""
+        B, n_pre, H, D = q_prefix.shape
+        pos = torch.from_numpy(self.prefix_positions()).to(self.device)
+        assert n_pre == pos.shape[1], "q_prefix must cover prompt + sink tokens"
+        lens = torch.tensor([p.lengths["prompt"] + p.lengths.get("sink", 0) for p in self.plans],
+                            dtype=torch.int32, device=self.device)
+        q_att = torch.empty(B, H, n_pre, D, dtype=torch.bfloat16, device=self.device)
+        o = torch.zeros(B, n_pre, H, D, dtype=torch.bfloat16, device=self.device)
+        lse = torch.empty(B, H, n_pre, dtype=torch.float32, device=self.device)
+        self.rotate_keys(stream)
+        self._rope(q_prefix, q_att.permute(0, 2, 1, 3), pos, key=False, n_valid=lens, stream=stream)
+        kv_len = self.kv_len.clone()
+        for si, name in enumerate(self.segments):
+            if name not in ("prompt", "sink"):
+                kv_len[:, si] = 0
+        ws_bytes = capi.sr_chunk_attention_workspace_bytes(B, H, D, n_pre)
+        ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=self.device) if ws_bytes else None
+        capi.sr_chunk_attention_fwd(q_att, self.k_att, self.v, o, lse, self.caps, kv_len, lens, self.scale,
+                                    self.status, workspace=ws, stream=stream)
+        self.prefix_lse = lse
+        return o
+
+    def step_moving(self, q_recent: torch.Tensor, k_recent: torch.Tensor, v_recent: torch.Tensor,
+                    q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream=None) -> torch.Tensor:
+        """The moving part of one denoising step: the recent frames' recomputed
+        K (before RoPE) and V replace the recent segment, the chunk's K and V
+        the chunk segment, and the queries of the recent frames followed by
+        the chunk attend to the whole window.  Recent tensors [B, n_recent,
+        H, D] (every session the same n_recent), chunk tensors as in step().
+        Returns o [B, n_recent + q_cap, H, D]."""
+        B, n_rec, H, D = q_recent.shape
+        off_r, _ = self.seg["recent"]
+        if any(p.lengths["recent"] != n_rec for p in self.plans):
+            raise ValueError("every session must hold n_recent recent tokens")
+        capi.sr_kv_append(self.k_raw, self.v, None, off_r, k_recent, v_recent, None, stream=stream)
+        self.append_chunk(k, v, stream)
+        self.rotate(q, stream)   # window keys + chunk queries (the latter reused below)
+        n_mov = n_rec + self.q_cap
+        q_att = torch.empty(B, H, n_mov, D, dtype=torch.bfloat16, device=self.device)
+        q_att[:, :, n_rec:].copy_(self.q_att)
+        pos_r = self.pos[:, off_r:off_r + n_rec]
+        self._rope(q_recent, q_att[:, :, :n_rec].permute(0, 2, 1, 3), pos_r, key=False, stream=stream)
+        o = torch.zeros(B, n_mov, H, D, dtype=torch.bfloat16, device=self.device)
+        lse = torch.empty(B, H, n_mov, dtype=torch.float32, device=self.device)
+        q_len = self.q_len + n_rec
+        ws_bytes = capi.sr_chunk_attention_workspace_bytes(B, H, D, n_mov)
+        ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=self.device) if ws_bytes else None
+        capi.sr_chunk_attention_fwd(q_att, self.k_att, self.v, o, lse, self.caps, self.kv_len, q_len, self.scale,
+                                    self.status, workspace=ws, stream=stream)
+        self.moving_lse = lse
+        return o
 
     def check_status(self) -> None:
         """Raise if a bounded wait inside the attention kernel gave up

@@ -8,7 +8,7 @@ import pytest
 from streaming_video_audio_b200 import capi
 
 EXPECTED = {"sr_version", "sr_get_last_error", "sr_rope3d_apply", "sr_history_compress", "sr_kv_append",
-            "sr_chunk_attention_fwd", "sr_chunk_attention_workspace_bytes"}
+            "sr_chunk_attention_fwd", "sr_chunk_attention_workspace_bytes", "sr_qknorm_rope3d_apply"}
 
 
 def test_header_declares_the_boundary():

@@ -269,3 +269,79 @@ def test_attention_repeated_launches_deterministic():
     for _ in range(10):
         o, l = _run_attention(q, k, v, caps, lens, q_len, use_workspace=False)
         assert torch.equal(o[0, :129], _run_attention(q, k, v, caps, lens, q_len, use_workspace=False)[0][0, :129])
+
+
+# ---------------------------------------------------------------- QK-norm + RoPE (fused)
+@pytest.mark.parametrize("D,split,H,N", [(128, (32, 48, 48), 40, 200), (64, (16, 24, 24), 5, 33),
+                                         (128, (32, 48, 48), 56, 3)])
+def test_qknorm_rope_matches_oracle(D, split, H, N):
+    B = 2
+    x = workloads.draw_tensor((B, N, H, D), seed=90, scale=3.0)
+    gamma = (1.0 + 0.1 * workloads.draw_tensor((D,), seed=91).float()).contiguous()
+    pos = torch.stack([workloads.draw_positions(N, seed=92 + b) for b in range(B)])
+    y = torch.zeros(B, H, N, D, dtype=torch.bfloat16, device=DEV)
+    y_raw = torch.zeros(B, N, H, D, dtype=torch.bfloat16, device=DEV)
+    capi.sr_qknorm_rope3d_apply(x.to(DEV), y.permute(0, 2, 1, 3), gamma.to(DEV), 1e-6, pos.to(DEV), split,
+                                y_raw=y_raw)
+    torch.cuda.synchronize()
+    for b in range(B):
+        u = oracle.rms_norm(x[b], gamma.double(), 1e-6)                  # [N, H, D]
+        assert ulp_diff_bf16(y_raw[b].cpu(), u).max() <= 1
+        ref = oracle.rope3d(u, pos[b].double(), split)
+        assert_rope_close(y[b].permute(1, 0, 2).cpu(), ref, torch.from_numpy(u))
+
+
+# ---------------------------------------------------------------- windowed attention (causal VAE decoder)
+@pytest.mark.parametrize("D,split,shift", [(64, (16, 24, 24), 0), (64, (16, 24, 24), 8), (128, (32, 48, 48), 8)])
+def test_ring_window_attention_matches_oracle(D, split, shift):
+    """Four calls of 2 latent frames through a 6-frame ring (empty, half-full,
+    full, wrapped) on a grid whose edge windows are partial."""
+    from oracle import vae_window
+    from streaming_video_audio_b200.vae_window import RingWindowAttention
+    gh, gw, H, calls = 20, 36, 2, 4
+    T = gh * gw
+    F = 2 * calls
+    q = workloads.draw_tensor((F, T, H, D), seed=100)
+    k = workloads.draw_tensor((F, T, H, D), seed=101)
+    v = workloads.draw_tensor((F, T, H, D), seed=102)
+    layer = RingWindowAttention((gh, gw), H, D, split, shift=shift)
+    t0 = 57                                     # stream clock of frame 0
+    for c in range(calls):
+        fr = slice(2 * c, 2 * c + 2)
+        o = layer(q[fr].reshape(2 * T, H, D).cuda(), k[fr].reshape(2 * T, H, D).cuda(),
+                  v[fr].reshape(2 * T, H, D).cuda(), t0=t0 + 2 * c)
+        torch.cuda.synchronize()
+        assert int(layer.status.item()) == 0
+        ref = vae_window.window_attention_reference(q[:2 * c + 2], k[:2 * c + 2], v[:2 * c + 2], (gh, gw), t0=t0,
+                                                    call_frames=2, history=4, split=split, shift=shift)
+        mx, mean = attn_errors(o.cpu(), ref)
+        assert mx <= ATTN_MAX_ABS and mean <= ATTN_MEAN_ABS, (c, mx, mean)
+
+
+def test_ring_window_attention_is_causal_and_clock_invariant():
+    """Changing a later call's frames leaves earlier outputs bit-identical, and
+    starting the stream clock elsewhere changes nothing but rounding."""
+    from streaming_video_audio_b200.vae_window import RingWindowAttention
+    gh, gw, H, D, T = 20, 36, 2, 64, 20 * 36
+    q = workloads.draw_tensor((6, T, H, D), seed=110)
+    k = workloads.draw_tensor((6, T, H, D), seed=111)
+    v = workloads.draw_tensor((6, T, H, D), seed=112)
+
+    def run(qq, kk, vv, t0):
+        layer = RingWindowAttention((gh, gw), H, D, (16, 24, 24), shift=8)
+        outs = []
+        for c in range(3):
+            fr = slice(2 * c, 2 * c + 2)
+            outs.append(layer(qq[fr].reshape(2 * T, H, D).cuda(), kk[fr].reshape(2 * T, H, D).cuda(),
+                              vv[fr].reshape(2 * T, H, D).cuda(), t0=t0 + 2 * c).cpu())
+        return outs
+
+    a = run(q, k, v, 0)
+    k2, v2 = k.clone(), v.clone()
+    k2[4:] = workloads.draw_tensor((2, T, H, D), seed=113)
+    v2[4:] = workloads.draw_tensor((2, T, H, D), seed=114)
+    b = run(q, k2, v2, 0)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1]) and not torch.equal(a[2], b[2])
+    c = run(q, k, v, 1000)
+    for x, y in zip(a, c):
+        assert float((x.float() - y.float()).abs().max()) <= 2e-2

@@ -110,3 +110,56 @@ def test_window_layout_matches_oracle(config):
                 assert np.array_equal(got_v.double().numpy(), seg["v"]), seg["name"]
         assert not win.v[b, :, torch.from_numpy(~mask).cuda()].any()
         assert not np.any(pos[b, ~mask])
+
+
+def test_step_with_qk_norm_matches_oracle():
+    """The layer with QK normalisation: keys are kept before normalisation,
+    pooled, then normalised and rotated in one fused kernel every step."""
+    spec = workloads.scaled(workloads.CHUNK_TIERED, n_heads=4, prompt_len=37, context_video_tokens=25 * 1008,
+                            chunk_video_tokens=1008 + 300, chunk_audio_tokens=20)
+    inp = workloads.draw_session(spec, 7)
+    gq = 1.0 + 0.2 * workloads.draw_tensor((128,), seed=8).float()
+    gk = 1.0 + 0.2 * workloads.draw_tensor((128,), seed=9).float()
+    win = StreamingWindow([spec], qk_norm=(gq, gk, 1e-6))
+    win.load_window([inp])
+    win.step(inp.q.cuda()[None], inp.k.cuda()[None], inp.v.cuda()[None])
+    torch.cuda.synchronize()
+    win.check_status()
+    rows = sample_rows(spec.chunk_len, 64, seed=3)
+    ref_o, _ = oracle.session_reference(spec, inp, rows=rows, qk_norm=(gq.double().numpy(), gk.double().numpy(), 1e-6))
+    o = win.o.cpu()
+    for h in range(spec.n_heads):
+        mx, mean = attn_errors(o[0, rows, h], ref_o[:, h])
+        assert mx <= ATTN_MAX_ABS and mean <= ATTN_MEAN_ABS, (h, mx, mean)
+
+
+@pytest.mark.parametrize("config", [2, 3])
+def test_prefix_self_and_moving_part_match_oracle(config):
+    """Prefix queries (prompt + sink) see only the prefix; recent + chunk
+    queries see the whole window with recomputed recent K/V; two denoising
+    steps are two banks (batch entries) with their own inputs."""
+    spec = workloads.scaled(workloads.CONFIGS[config], n_heads=3)
+    seeds = [11, 12]                                # one bank per denoising step
+    inputs = [workloads.draw_session(spec, s) for s in seeds]
+    movs = [workloads.draw_moving(spec, s) for s in seeds]
+    win = StreamingWindow([spec, spec])
+    win.load_window(inputs)
+    stack = lambda name, src: torch.stack([getattr(x, name) for x in src]).cuda()
+    o_pre = win.attend_prefix(stack("prefix_q", movs))
+    o_mov = win.step_moving(stack("recent_q", movs), stack("recent_k", movs), stack("recent_v", movs),
+                            stack("q", inputs), stack("k", inputs), stack("v", inputs))
+    torch.cuda.synchronize()
+    win.check_status()
+    n_pre = spec.prompt_len + workloads.sink_tokens(spec)
+    n_mov = workloads.recent_tokens(spec) + spec.chunk_len
+    for b in range(2):
+        rows = sample_rows(n_pre, 32, seed=b)
+        ref, _ = oracle.prefix_reference(spec, inputs[b], movs[b], rows=rows)
+        for h in range(3):
+            mx, mean = attn_errors(o_pre[b, rows, h].cpu(), ref[:, h])
+            assert mx <= ATTN_MAX_ABS and mean <= ATTN_MEAN_ABS, ("prefix", b, h, mx, mean)
+        rows = sample_rows(n_mov, 48, seed=10 + b)
+        ref, _ = oracle.moving_reference(spec, inputs[b], movs[b], rows=rows)
+        for h in range(3):
+            mx, mean = attn_errors(o_mov[b, rows, h].cpu(), ref[:, h])
+            assert mx <= ATTN_MAX_ABS and mean <= ATTN_MEAN_ABS, ("moving", b, h, mx, mean)

@@ -128,3 +128,30 @@ def test_session_reference_matches_sdpa_composition():
                                         sp.rope_split)).permute(1, 0, 2)
     ref = torch.nn.functional.scaled_dot_product_attention(qr, kr, torch.from_numpy(v).permute(1, 0, 2))
     np.testing.assert_allclose(o, ref.permute(1, 0, 2).numpy()[rows], atol=1e-12)
+
+
+def test_prefix_and_moving_references_reduce_to_plain_attention():
+    """The prefix-self attention equals plain attention of the prefix queries
+    over [prompt | sink] keys; the moving-part attention of the chunk rows
+    equals the whole-step reference once the recent frames' K/V are swapped
+    for the recomputed ones; without a prefix-only mask the prefix rows would
+    differ (the mask matters)."""
+    sp = workloads.scaled(workloads.TINY, prompt_len=5)
+    inp = workloads.draw_session(sp, 2)
+    mov = workloads.draw_moving(sp, 2)
+    o_pre, l_pre = oracle.prefix_reference(sp, inp, mov)
+    segs = {s["name"]: s for s in oracle.session_kv(sp, inp)}
+    k = np.concatenate([segs["prompt"]["k"], segs["sink"]["k"]])[:, 0]
+    v = np.concatenate([segs["prompt"]["v"], segs["sink"]["v"]])[:, 0]
+    p = np.concatenate([segs["prompt"]["pos"], segs["sink"]["pos"]])
+    kr = torch.from_numpy(oracle.rope3d(k, p, sp.rope_split))[None]
+    qr = torch.from_numpy(oracle.rope3d(mov.prefix_q[:, 0].double().numpy(), p, sp.rope_split))[None]
+    ref = torch.nn.functional.scaled_dot_product_attention(qr, kr, torch.from_numpy(v)[None])[0].numpy()
+    np.testing.assert_allclose(o_pre[:, 0], ref, atol=1e-12)
+    # moving part: the chunk rows see the recomputed recent frames
+    o_mov, _ = oracle.moving_reference(sp, inp, mov)
+    assert o_mov.shape[0] == workloads.recent_tokens(sp) + sp.chunk_len
+    inp2 = workloads.SessionInputs(inp.prompt_k, inp.prompt_v, inp.ctx_k[:1] + [mov.recent_k], inp.ctx_v[:1] + [mov.recent_v],
+                                   inp.q, inp.k, inp.v)
+    o_step, _ = oracle.session_reference(sp, inp2)
+    np.testing.assert_allclose(o_mov[workloads.recent_tokens(sp):], o_step, atol=1e-12)

@@ -124,3 +124,36 @@ def test_session_kv_places_input_tokens():
     assert by["chunk"]["pos"][2 * 1008 + 4].tolist() == [2.0, 0.0, 4.0]
     assert by["tier1"]["pos"][0].tolist() == [-12.0, 0.5, 0.5]
     assert by["tier0"]["pos"][65].tolist() == [-24.0, 21.5, 40.5]
+
+
+def test_window_reference_reduces_to_full_attention_when_one_window_covers_the_grid():
+    """A grid smaller than one window with no shift: every token of the
+    history range is in the single window, so the reference is plain
+    attention of the current frames over all kept frames."""
+    from oracle import vae_window
+    F, gh, gw, H, D = 5, 6, 7, 1, 64
+    q = workloads.draw_tensor((F, gh * gw, H, D), seed=1)
+    k = workloads.draw_tensor((F, gh * gw, H, D), seed=2)
+    v = workloads.draw_tensor((F, gh * gw, H, D), seed=3)
+    o = vae_window.window_attention_reference(q, k, v, (gh, gw), t0=10, call_frames=2, history=2,
+                                              split=(16, 24, 24))
+    kept = list(range(1, 5))                      # frames 3, 4 current + 2 of history
+    rr, cc = np.divmod(np.arange(gh * gw), gw)
+    pos = lambda fs: np.concatenate([np.stack([np.full(gh * gw, 10 + f), rr, cc], 1) for f in fs]).astype(float)
+    kr = oracle.rope3d(k[kept, :, 0].reshape(-1, D), pos(kept), (16, 24, 24))
+    qr = oracle.rope3d(q[[3, 4], :, 0].reshape(-1, D), pos([3, 4]), (16, 24, 24))
+    ref = torch.nn.functional.scaled_dot_product_attention(torch.from_numpy(qr)[None], torch.from_numpy(kr)[None],
+                                                           v[kept, :, 0].reshape(-1, D).double()[None])[0]
+    np.testing.assert_allclose(o[:, 0], ref.numpy(), atol=1e-12)
+
+
+def test_window_membership_partitions_the_grid():
+    from oracle import vae_window
+    for shift in (0, 8):
+        seen = {}
+        for r in range(20):
+            for c in range(36):
+                seen.setdefault(vae_window.window_of(r, c, 16, shift), []).append((r, c))
+        assert sum(len(x) for x in seen.values()) == 20 * 36
+        assert all(len(x) <= 256 for x in seen.values())
+        assert len(seen) == (-(-(20 + shift) // 16)) * (-(-(36 + shift) // 16))

@@ -190,3 +190,35 @@ def draw_positions(n: int, seed: int, spread: float = 32.0) -> torch.Tensor:
     """Seeded fp32 (t, h, w) positions, uniform in [-spread, spread)."""
     x = np.random.default_rng(seed).uniform(-spread, spread, size=(n, 3)).astype(np.float32)
     return torch.from_numpy(x)
+
+
+@dataclasses.dataclass
+class MovingInputs:
+    """Extra bf16 tensors for the prefix / moving-part split of a window:
+    queries of the fixed prefix (prompt then sink tokens) and recomputed
+    queries, keys and values of the recent frames (token-major [L, H, D])."""
+    prefix_q: torch.Tensor
+    recent_q: torch.Tensor
+    recent_k: torch.Tensor
+    recent_v: torch.Tensor
+
+
+def recent_tokens(spec: SessionSpec) -> int:
+    """Full-resolution context tokens after the sink and the pooled tiers."""
+    sizes = spec.context_frame_tokens()
+    skip = min(spec.sink_frames, len(sizes)) + sum(n for n, _, _ in spec.tiers)
+    return sum(sizes[skip:])
+
+
+def sink_tokens(spec: SessionSpec) -> int:
+    return sum(spec.context_frame_tokens()[:spec.sink_frames])
+
+
+def draw_moving(spec: SessionSpec, seed: int) -> MovingInputs:
+    """Drawn from default_rng([seed, 1]) in this order: prefix Q, recent Q,
+    recent K, recent V (same distribution as the session's tensors)."""
+    rng = np.random.default_rng([seed, 1])
+    n_prefix = spec.prompt_len + sink_tokens(spec)
+    n_recent = recent_tokens(spec)
+    return MovingInputs(_draw(rng, n_prefix, spec), _draw(rng, n_recent, spec), _draw(rng, n_recent, spec),
+                        _draw(rng, n_recent, spec))
