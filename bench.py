@@ -327,22 +327,29 @@ def main():
     total_ms = start.elapsed_time(stop)
     attn_ms = [a.elapsed_time(b) for a, b in evs]
 
-    # end to end through the public host-buffer API
+    # end to end through the public host-buffer API: every step uploads its
+    # q, k, v from pinned host memory and downloads its o; HostStepPipeline
+    # overlaps those transfers with the neighbouring steps' compute
+    from streaming_video_audio_b200.window import HostStepPipeline
     qh, kh, vh = (t.pin_memory() for t in chunk)
-    oh = torch.empty(win.o.shape, dtype=torch.bfloat16).pin_memory()
-    staging = tuple(torch.empty_like(t, device=device) for t in chunk)
+    ohs = [torch.empty(win.o.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    pipe = HostStepPipeline(win)
     for i in range(W):
-        win.step_from_host(qh, kh, vh, oh, staging)
-    torch.cuda.synchronize()
+        pipe.step(qh, kh, vh, ohs[i % 2])
+    pipe.synchronize()
     if dist:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
     e0.record(stream)
     for i in range(K):
-        win.step_from_host(qh, kh, vh, oh, staging)
+        pipe.step(qh, kh, vh, ohs[i % 2])
+    stream.wait_stream(pipe.copy)
+    stream.wait_stream(pipe.copy_back)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
+    oh = ohs[0]
     if dist:
         dist.barrier()
 

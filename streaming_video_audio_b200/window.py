@@ -264,18 +264,21 @@ class StreamingWindow:
             capi.sr_qknorm_rope3d_apply(x, y, gk if key else gq, eps, pos, self.split, self.base, n_valid=n_valid,
                                         stream=stream)
 
-    def attend(self, stream=None) -> torch.Tensor:
-        """a4: fused chunk attention -> o [B, q_cap, H, D] (and lse)."""
-        capi.sr_chunk_attention_fwd(self.q_att, self.k_att, self.v, self.o, self.lse, self.caps, self.kv_len,
+    def attend(self, stream=None, out: torch.Tensor = None) -> torch.Tensor:
+        """a4: fused chunk attention -> o [B, q_cap, H, D] (and lse); `out`
+        optionally replaces the window's own output buffer."""
+        o = self.o if out is None else out
+        capi.sr_chunk_attention_fwd(self.q_att, self.k_att, self.v, o, self.lse, self.caps, self.kv_len,
                                     self.q_len, self.scale, self.status, workspace=self.workspace, stream=stream)
-        return self.o
+        return o
 
-    def step(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream=None) -> torch.Tensor:
+    def step(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream=None,
+             out: torch.Tensor = None) -> torch.Tensor:
         """One streaming attention step: a2 -> a3 -> a4 (device tensors
         [B, q_cap, H, D], token-major, pre-RoPE)."""
         self.append_chunk(k, v, stream)
         self.rotate(q, stream)
-        return self.attend(stream)
+        return self.attend(stream, out=out)
 
     def step_from_host(self, q_host: torch.Tensor, k_host: torch.Tensor, v_host: torch.Tensor,
                        o_host: torch.Tensor, staging=None, stream=None) -> torch.Tensor:
@@ -416,3 +419,53 @@ class StreamingWindow:
             capi.sr_history_compress(frames(self.k_raw, so, src_tok), frames(self.v, so, src_tok),
                                      frames(self.k_raw, do, dst_tok), frames(self.v, do, dst_tok),
                                      (gh, gw), (ph, pw), stream=stream)
+
+
+class HostStepPipeline:
+    """Runs consecutive streaming steps for a caller that holds its tensors in
+    pinned host memory, overlapping the transfers with the compute: step i+1's
+    uploads and step i's download run on a copy stream while step i computes
+    on the compute stream.  Two staging sets (q, k, v, o) alternate between
+    steps; every step still moves its own inputs and its output.
+
+        pipe = HostStepPipeline(window)
+        for q_h, k_h, v_h, o_h in steps:          # pinned host tensors
+            pipe.step(q_h, k_h, v_h, o_h)           # asynchronous
+        pipe.synchronize()                          # every o_h is now valid
+    """
+
+    def __init__(self, window: StreamingWindow, depth: int = 2):
+        self.win = window
+        dev = window.device
+        shape = (window.B, window.q_cap, window.H, window.D)
+        self.compute = torch.cuda.current_stream(dev)
+        self.copy = torch.cuda.Stream(device=dev)       # uploads
+        self.copy_back = torch.cuda.Stream(device=dev)  # downloads (the link is full duplex)
+        self.sets = [tuple(torch.empty(shape, dtype=torch.bfloat16, device=dev) for _ in range(4))
+                     for _ in range(depth)]
+        self.free = [torch.cuda.Event() for _ in range(depth)]   # staging set reusable (its download done)
+        self.i = 0
+
+    def step(self, q_h: torch.Tensor, k_h: torch.Tensor, v_h: torch.Tensor, o_h: torch.Tensor) -> None:
+        s = self.i % len(self.sets)
+        q, k, v, o = self.sets[s]
+        uploaded, computed = torch.cuda.Event(), torch.cuda.Event()
+        with torch.cuda.stream(self.copy):
+            self.copy.wait_event(self.free[s])
+            q.copy_(q_h, non_blocking=True)
+            k.copy_(k_h, non_blocking=True)
+            v.copy_(v_h, non_blocking=True)
+            uploaded.record(self.copy)
+        self.compute.wait_event(uploaded)
+        self.win.step(q, k, v, stream=self.compute, out=o)
+        computed.record(self.compute)
+        with torch.cuda.stream(self.copy_back):
+            self.copy_back.wait_event(computed)
+            o_h.copy_(o, non_blocking=True)
+            self.free[s].record(self.copy_back)
+        self.i += 1
+
+    def synchronize(self) -> None:
+        self.copy.synchronize()
+        self.copy_back.synchronize()
+        self.compute.synchronize()

@@ -163,3 +163,27 @@ def test_prefix_self_and_moving_part_match_oracle(config):
         for h in range(3):
             mx, mean = attn_errors(o_mov[b, rows, h].cpu(), ref[:, h])
             assert mx <= ATTN_MAX_ABS and mean <= ATTN_MEAN_ABS, ("moving", b, h, mx, mean)
+
+
+def test_host_step_pipeline_matches_device_step():
+    """The pipelined host-buffer path returns, for every step, exactly the
+    output of the device step on the same inputs."""
+    from streaming_video_audio_b200.window import HostStepPipeline
+    spec = workloads.scaled(workloads.CHUNK, n_heads=4)
+    inp = workloads.draw_session(spec, 4)
+    win = StreamingWindow([spec])
+    win.load_window([inp])
+    chunks = []
+    for s in range(3):
+        x = workloads.draw_session(spec, 50 + s)
+        chunks.append(tuple(getattr(x, n)[None].contiguous() for n in ("q", "k", "v")))
+    refs = []
+    for q, k, v in chunks:
+        refs.append(win.step(q.cuda(), k.cuda(), v.cuda()).cpu().clone())
+    pipe = HostStepPipeline(win)
+    outs = [torch.empty_like(r).pin_memory() for r in refs]
+    for (q, k, v), o in zip(chunks, outs):
+        pipe.step(q.pin_memory(), k.pin_memory(), v.pin_memory(), o)
+    pipe.synchronize()
+    for r, o in zip(refs, outs):
+        assert torch.equal(r, o)
