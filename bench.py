@@ -3,9 +3,10 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config {2,3,4,5}] [--impl {sr,reference}]
 
 A step is one pass of the whole hot path on one batch of synthetic inputs
-resident in HBM: history-tier pooling of the frames that cross a tier
-boundary (a1, configs with tiers), KV append of the chunk (a2), RoPE of the
-chunk queries and of every window key (a3) and the fused chunk attention
+resident in HBM: the window slide of the tiered configs (a1: the frames that
+cross a tier boundary are pooled into the older tier and the previous chunk's
+clean frames become the recent ones), KV append of the chunk (a2), RoPE of
+the chunk queries and of every window key (a3) and the fused chunk attention
 (a4).  Default workload: the tiered streaming chunk (config 3), the one
 config on which all four steps run.
 
@@ -180,11 +181,16 @@ def attention_traffic(config: int):
     return int(rec["dram_bytes_read"]) + int(rec["dram_bytes_write"])
 
 
-def launches_per_step(win, tiered: bool) -> int:
-    # append, RoPE of q, RoPE of the window, attention (+ the split merge)
-    n = 4 + (1 if win.workspace is not None else 0)
+def launches_in_steps(win, tiered: bool, steps: int) -> int:
+    """Library kernel launches of `steps` steps from the window's current
+    slide state: append, RoPE of q, RoPE of the window, attention (+ the
+    split merge) per step, and the slide's pooling and append calls."""
+    n = (4 + (1 if win.workspace is not None else 0)) * steps
     if tiered:
-        n += len(win.tier_boundaries())
+        ptr = dict(win.ring_ptr)
+        for _ in range(steps):
+            ops, ptr = win.slide_ops(ptr)
+            n += len(ops)
     return n
 
 
@@ -293,9 +299,12 @@ def main():
     stream = torch.cuda.current_stream()
     K, W = args.steps, args.warmup
 
+    n_video = specs[0].chunk_video_tokens
+    k_clean, v_clean = k[:, :n_video], v[:, :n_video]   # stand-in for the finished chunk's clean K/V
+
     def one_step(i, ev=None):
         if tiered:
-            win.age_tiers(i, 3)
+            win.advance(k_clean, v_clean)
         win.append_chunk(k, v)
         win.rotate(q)
         if ev is not None:
@@ -309,6 +318,7 @@ def main():
     torch.cuda.synchronize()
     win.check_status()
 
+    launches = launches_in_steps(win, tiered, K)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local)
@@ -329,13 +339,14 @@ def main():
 
     # end to end through the public host-buffer API: every step uploads its
     # q, k, v from pinned host memory and downloads its o; HostStepPipeline
-    # overlaps those transfers with the neighbouring steps' compute
+    # overlaps those transfers with the neighbouring steps' compute; the
+    # slide takes the previous step's uploaded chunk as the clean frames
     from streaming_video_audio_b200.window import HostStepPipeline
     qh, kh, vh = (t.pin_memory() for t in chunk)
     ohs = [torch.empty(win.o.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
     pipe = HostStepPipeline(win)
     for i in range(W):
-        pipe.step(qh, kh, vh, ohs[i % 2])
+        pipe.step(qh, kh, vh, ohs[i % 2], slide=tiered)
     pipe.synchronize()
     if dist:
         dist.barrier()
@@ -343,7 +354,7 @@ def main():
     torch.cuda.synchronize()
     e0.record(stream)
     for i in range(K):
-        pipe.step(qh, kh, vh, ohs[i % 2])
+        pipe.step(qh, kh, vh, ohs[i % 2], slide=tiered)
     stream.wait_stream(pipe.copy)
     stream.wait_stream(pipe.copy_back)
     e1.record(stream)
@@ -384,7 +395,7 @@ def main():
                     "h2d_bytes_per_step": sum(t.numel() * 2 for t in chunk),
                     "d2h_bytes_per_step": oh.numel() * 2},
             "clocks": clocks,
-            "gpu_launches": launches_per_step(win, tiered) * K,
+            "gpu_launches": launches,
         }
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(specs, inputs)

@@ -139,4 +139,5 @@ def attention(q, k, v, scale: float, rows: Optional[Sequence[int]] = None):
 
 
 from . import layout  # noqa: E402  (layout needs nothing above but keeps the public surface here)
-from .session import session_reference, session_kv, pooled_tier, prefix_reference, moving_reference  # noqa: E402,F401
+from .session import (session_reference, session_kv, pooled_tier, prefix_reference, moving_reference,  # noqa: E402,F401
+                      slide_window)

@@ -176,3 +176,26 @@ def moving_reference(spec, inp, mov, heads: Optional[Sequence[int]] = None, rows
         o[:, hi], lse[:, hi] = attention(np.ascontiguousarray(q_rot[:, hi]), np.ascontiguousarray(k_rot[:, hi]),
                                          np.ascontiguousarray(v[:, hi]), scale)
     return o, lse
+
+
+def slide_window(spec, inp, clean_k, clean_v, q, k, v):
+    """The session one chunk later: the finished chunk's clean video frames
+    (token-major [n * Gh*Gw, H, D]) join the history as its newest frames,
+    the n oldest frames after the sink leave it, and the next chunk's q, k, v
+    replace the chunk.  Every tier is then pooled afresh from full resolution
+    by ``session_kv`` (the definition of the window at that time).
+
+    Reading: "StreamRender-H3" (molayo1419.me), streaming context section --
+    the context is the sink plus the most recent outputs, so a finished chunk
+    pushes the oldest non-sink frames out; "AlayaRenderer-Flash"
+    (aitrends.kr), technical details -- frames age from the recent tier into
+    the pooled tiers, oldest tier coarsest."""
+    ft = spec.grid_h * spec.grid_w
+    n = clean_k.shape[0] // ft
+    assert n * ft == clean_k.shape[0] and clean_v.shape == clean_k.shape
+    sink = spec.sink_frames
+    hist_k = list(inp.ctx_k[sink:]) + [clean_k[i * ft:(i + 1) * ft] for i in range(n)]
+    hist_v = list(inp.ctx_v[sink:]) + [clean_v[i * ft:(i + 1) * ft] for i in range(n)]
+    keep = len(inp.ctx_k) - sink
+    return type(inp)(inp.prompt_k, inp.prompt_v, list(inp.ctx_k[:sink]) + hist_k[-keep:],
+                     list(inp.ctx_v[:sink]) + hist_v[-keep:], q, k, v)

@@ -193,6 +193,9 @@ class StreamingWindow:
         lists of [tokens, H, D] full-resolution frames, oldest first).  Tier
         frames are pooled on the device by sr_history_compress."""
         dev = self.device
+        if hasattr(self, "rings"):   # a reload restarts the window slide
+            self.pos = self._pos_loaded
+            del self.rings
         for b, (plan, inp) in enumerate(zip(self.plans, inputs)):
             kb, vb, pb = self.k_raw[b:b + 1], self.v[b:b + 1], self.pos[b:b + 1]
             lp = plan.lengths["prompt"]
@@ -350,13 +353,30 @@ class StreamingWindow:
         off_r, _ = self.seg["recent"]
         if any(p.lengths["recent"] != n_rec for p in self.plans):
             raise ValueError("every session must hold n_recent recent tokens")
-        capi.sr_kv_append(self.k_raw, self.v, None, off_r, k_recent, v_recent, None, stream=stream)
+        # after window slides the recent frames sit in ring order: write each
+        # run of consecutive slots with one append, read positions likewise
+        ft = self.plans[0].frame_tokens
+        order = self.recent_slot_order()
+        runs, j = [], 0
+        while j < len(order):
+            m = 1
+            while j + m < len(order) and order[j + m] == order[j] + m:
+                m += 1
+            runs.append((order[j], j, m))
+            j += m
+        for slot, j, m in runs:
+            rows = slice(j * ft, min((j + m) * ft, n_rec))
+            capi.sr_kv_append(self.k_raw, self.v, None, off_r + slot * ft, k_recent[:, rows], v_recent[:, rows],
+                              None, stream=stream)
         self.append_chunk(k, v, stream)
         self.rotate(q, stream)   # window keys + chunk queries (the latter reused below)
         n_mov = n_rec + self.q_cap
         q_att = torch.empty(B, H, n_mov, D, dtype=torch.bfloat16, device=self.device)
         q_att[:, :, n_rec:].copy_(self.q_att)
-        pos_r = self.pos[:, off_r:off_r + n_rec]
+        if len(runs) == 1:
+            pos_r = self.pos[:, off_r:off_r + n_rec]
+        else:   # a wrapped ring holds whole frames only
+            pos_r = torch.cat([self.pos[:, off_r + slot * ft:off_r + (slot + m) * ft] for slot, _, m in runs], dim=1)
         self._rope(q_recent, q_att[:, :, :n_rec].permute(0, 2, 1, 3), pos_r, key=False, stream=stream)
         o = torch.zeros(B, n_mov, H, D, dtype=torch.bfloat16, device=self.device)
         lse = torch.empty(B, H, n_mov, dtype=torch.float32, device=self.device)
@@ -376,7 +396,6 @@ class StreamingWindow:
             self.status.zero_()
             raise capi.SrError("sr_chunk_attention_fwd", s, "a pipeline wait timed out on the device")
 
-    # ---------------------------------------------------------------- tier aging
     def tier_boundaries(self):
         """(source segment, destination tier, source grid, pool) for every tier
         boundary, destination-oldest first: each tier is fed by the next
@@ -395,31 +414,156 @@ class StreamingWindow:
             out.append((src, dst, (gh, gw), (_ceil_div(gh, dh), _ceil_div(gw, dw))))
         return out
 
-    def age_tiers(self, step_index: int, n_frames: int, stream=None) -> None:
-        """a1 in steady-state streaming: at every tier boundary the n_frames
-        oldest frames of the newer segment are pooled into the older tier
-        (oldest boundary first, so a tier's frames are consumed before they
-        are overwritten).  Frames live in ring slots that advance with
-        step_index; segment lengths stay constant (full rings).  K and V are
-        pooled pre-RoPE; positions are rewritten by the next re-positioning."""
-        for src, dst, (gh, gw), (ph, pw) in self.tier_boundaries():
-            src_tok = gh * gw
-            dst_tok = _ceil_div(gh, ph) * _ceil_div(gw, pw)
-            n_src = self.plans[0].lengths[src] // src_tok
-            n_dst = self.plans[0].lengths[dst] // dst_tok
-            fs = (step_index * n_frames) % n_src
-            fd = (step_index * n_frames) % n_dst
-            nf = min(n_frames, n_src - fs, n_dst - fd)
-            so = self.seg[src][0] + fs * src_tok
-            do = self.seg[dst][0] + fd * dst_tok
+    # ---------------------------------------------------------------- window slide
+    # After a chunk is finished its clean frames become the newest context;
+    # every tier hands its oldest frames to the next older tier, pooled once
+    # more, and the oldest tier drops its oldest frames.  The sink stays.
+    # Each of tier0.., recent is a ring of frame slots with a pointer to its
+    # oldest frame, so nothing is moved but the frames that change tier; the
+    # window template (t of a frame = its rank in the window) is rewritten by
+    # switching to a precomputed position table of the new ring state.
+    MAX_PHASES = 64
 
-            def frames(buf, off, tok):
-                return buf[:, :, off:off + nf * tok].permute(0, 2, 1, 3).reshape(self.B, nf, tok, self.H, self.D)
+    def _ring_setup(self, n: int) -> None:
+        """Host side of the rings for slides of n frames: per ring its slot
+        count, tokens per frame, template t of its oldest frame; the pointer
+        state starts at 0 (load_window fills slots in chronological order)."""
+        plan = self.plans[0]
+        if any(p.context != plan.context for p in self.plans):
+            raise ValueError("the window slide needs sessions with the same context structure")
+        rings = {}
+        for role, t, ph, pw, ntok in plan.context:
+            if role == "sink":
+                continue
+            if ntok != plan.frame_tokens:
+                raise ValueError("the window slide needs whole history frames")
+            tok = plan.cells(ph, pw) if role.startswith("tier") else plan.frame_tokens
+            r = rings.setdefault(role, {"frames": 0, "tok": tok, "t0": t})
+            r["frames"] += 1
+        if "recent" not in rings or any(n > r["frames"] for r in rings.values()):
+            raise ValueError(f"a slide of {n} frames must fit in every history ring "
+                             f"({ {k: r['frames'] for k, r in rings.items()} })")
+        self.rings, self.slide_frames = rings, n
+        self.ring_ptr = {k: 0 for k in rings}
+        # each pointer moves n slots per slide: F / gcd(F, n) states per ring
+        self.period = math.lcm(*[r["frames"] // math.gcd(r["frames"], n) for r in rings.values()])
 
-            capi.sr_history_compress(frames(self.k_raw, so, src_tok), frames(self.v, so, src_tok),
-                                     frames(self.k_raw, do, dst_tok), frames(self.v, do, dst_tok),
-                                     (gh, gw), (ph, pw), stream=stream)
+    def ring_positions(self, ptr) -> np.ndarray:
+        """[cap_total, 3] template positions of the history ring slots for
+        pointer state ``ptr`` (other rows zero): t from the frame's rank in its
+        ring, (h, w) its grid cell or its cell's member mean."""
+        plan = self.plans[0]
+        pos = np.zeros((self.cap_total, 3), dtype=np.float32)
+        for role, r in self.rings.items():
+            off = self.seg[role][0]
+            if role.startswith("tier"):
+                _, ph, pw = plan.spec.tiers[int(role[4:])]
+                cells = []
+                for ci in range(_ceil_div(plan.gh, ph)):
+                    for cj in range(_ceil_div(plan.gw, pw)):
+                        r0, r1 = ci * ph, min((ci + 1) * ph, plan.gh)
+                        c0, c1 = cj * pw, min((cj + 1) * pw, plan.gw)
+                        cells.append((0.5 * (r0 + r1 - 1), 0.5 * (c0 + c1 - 1)))
+                hw = np.asarray(cells, dtype=np.float32)
+            else:
+                hw = plan.grid_positions(0.0, plan.frame_tokens)[:, 1:]
+            for slot in range(r["frames"]):
+                rank = (slot - ptr[role]) % r["frames"]
+                rows = slice(off + slot * r["tok"], off + (slot + 1) * r["tok"])
+                pos[rows, 0] = r["t0"] + rank
+                pos[rows, 1:] = hw
+        return pos
 
+    def slide_ops(self, ptr):
+        """Kernel calls of one slide from pointer state ``ptr`` (host only):
+        ("pool", src, src_frame, dst, dst_frame, m, grid, pool) and
+        ("append", recent_frame, clean_frame, m), in launch order, and the
+        next pointer state.  Boundaries run oldest tier first, so a ring's
+        oldest frames are read before the next boundary overwrites them."""
+        n = self.slide_frames
+        ops, nxt = [], dict(ptr)
+        for src, dst, grid, pool in self.tier_boundaries():
+            rs, rd = self.rings[src], self.rings[dst]
+            done = 0
+            while done < n:   # split where either ring wraps around
+                fs = (ptr[src] + done) % rs["frames"]
+                fd = (ptr[dst] + done) % rd["frames"]
+                m = min(n - done, rs["frames"] - fs, rd["frames"] - fd)
+                ops.append(("pool", src, fs, dst, fd, m, grid, pool))
+                done += m
+            nxt[dst] = (ptr[dst] + n) % rd["frames"]
+        rr = self.rings["recent"]
+        done = 0
+        while done < n:
+            fr = (ptr["recent"] + done) % rr["frames"]
+            m = min(n - done, rr["frames"] - fr)
+            ops.append(("append", fr, done, m))
+            done += m
+        nxt["recent"] = (ptr["recent"] + n) % rr["frames"]
+        return ops, nxt
+
+    def _ring_frames(self, buf, role: str, first: int, n: int) -> torch.Tensor:
+        """[B, n, tok, H, D] view of n consecutive frame slots of a ring."""
+        r = self.rings[role]
+        off = self.seg[role][0] + first * r["tok"]
+        return buf[:, :, off:off + n * r["tok"]].permute(0, 2, 1, 3).reshape(self.B, n, r["tok"], self.H, self.D)
+
+    def _phase_tables(self) -> None:
+        """Device position tables of every pointer state the slides cycle
+        through (the sink, prompt and chunk rows copied from the loaded window)."""
+        if self.period > self.MAX_PHASES:
+            raise ValueError(f"ring period {self.period} > {self.MAX_PHASES} position tables")
+        ctx = [self.seg[r] for r in self.rings]
+        lo, hi = min(o for o, _ in ctx), max(o + c for o, c in ctx)
+        self._pos_loaded = self.pos
+        self._phases, ptr = {}, dict(self.ring_ptr)
+        for _ in range(self.period):
+            tab = self._pos_loaded.clone()
+            tab[:, lo:hi] = torch.from_numpy(self.ring_positions(ptr)[lo:hi]).to(self.device)
+            self._phases[tuple(ptr.values())] = tab
+            ptr = self.slide_ops(ptr)[1]
+
+    def advance(self, k_clean: torch.Tensor, v_clean: torch.Tensor, stream=None) -> None:
+        """Slide the window by the finished chunk (a1 in streaming use).
+
+        k_clean, v_clean: the chunk's clean video frames, token-major
+        [B, n * frame_tokens, H, D], K before RoPE (every session the same n,
+        at most every ring's frame count).  Launches one
+        sr_history_compress per tier boundary (two where a ring wraps) and
+        one sr_kv_append (two on a wrap); positions switch to the new state's
+        table (no copy); the next rotate() re-positions the keys."""
+        plan = self.plans[0]
+        n = k_clean.shape[1] // plan.frame_tokens
+        if n < 1 or n * plan.frame_tokens != k_clean.shape[1] or v_clean.shape != k_clean.shape:
+            raise ValueError("clean K/V must hold whole frames")
+        if not hasattr(self, "rings"):
+            self._ring_setup(n)
+            self._phase_tables()
+        elif n != self.slide_frames:
+            raise ValueError(f"every slide must move {self.slide_frames} frames")
+        ops, nxt = self.slide_ops(self.ring_ptr)
+        for op in ops:
+            if op[0] == "pool":
+                _, src, fs, dst, fd, m, grid, pool = op
+                capi.sr_history_compress(self._ring_frames(self.k_raw, src, fs, m),
+                                         self._ring_frames(self.v, src, fs, m),
+                                         self._ring_frames(self.k_raw, dst, fd, m),
+                                         self._ring_frames(self.v, dst, fd, m), grid, pool, stream=stream)
+            else:
+                _, fr, fc, m = op
+                ft = plan.frame_tokens
+                capi.sr_kv_append(self.k_raw, self.v, None, self.seg["recent"][0] + fr * ft,
+                                  k_clean[:, fc * ft:(fc + m) * ft], v_clean[:, fc * ft:(fc + m) * ft], None,
+                                  stream=stream)
+        self.ring_ptr = nxt
+        self.pos = self._phases[tuple(nxt.values())]
+
+    def recent_slot_order(self) -> List[int]:
+        """Recent frames in chronological order -> their ring slots."""
+        if not hasattr(self, "rings"):
+            return list(range(_ceil_div(self.plans[0].lengths.get("recent", 0), self.plans[0].frame_tokens)))
+        r = self.rings["recent"]
+        return [(self.ring_ptr["recent"] + j) % r["frames"] for j in range(r["frames"])]
 
 class HostStepPipeline:
     """Runs consecutive streaming steps for a caller that holds its tensors in
@@ -432,6 +576,10 @@ class HostStepPipeline:
         for q_h, k_h, v_h, o_h in steps:          # pinned host tensors
             pipe.step(q_h, k_h, v_h, o_h)           # asynchronous
         pipe.synchronize()                          # every o_h is now valid
+
+    With ``slide=True`` every step after the first first slides the window
+    by the previous step's chunk: the video rows of its K and V (already on
+    the device in the previous staging set) become the newest history.
     """
 
     def __init__(self, window: StreamingWindow, depth: int = 2):
@@ -444,19 +592,28 @@ class HostStepPipeline:
         self.sets = [tuple(torch.empty(shape, dtype=torch.bfloat16, device=dev) for _ in range(4))
                      for _ in range(depth)]
         self.free = [torch.cuda.Event() for _ in range(depth)]   # staging set reusable (its download done)
+        self.read = [torch.cuda.Event() for _ in range(depth)]   # ... and the slide after it has read its K, V
         self.i = 0
 
-    def step(self, q_h: torch.Tensor, k_h: torch.Tensor, v_h: torch.Tensor, o_h: torch.Tensor) -> None:
+    def step(self, q_h: torch.Tensor, k_h: torch.Tensor, v_h: torch.Tensor, o_h: torch.Tensor,
+             slide: bool = False) -> None:
         s = self.i % len(self.sets)
         q, k, v, o = self.sets[s]
         uploaded, computed = torch.cuda.Event(), torch.cuda.Event()
         with torch.cuda.stream(self.copy):
             self.copy.wait_event(self.free[s])
+            self.copy.wait_event(self.read[s])
             q.copy_(q_h, non_blocking=True)
             k.copy_(k_h, non_blocking=True)
             v.copy_(v_h, non_blocking=True)
             uploaded.record(self.copy)
         self.compute.wait_event(uploaded)
+        if slide and self.i > 0:
+            p = (self.i - 1) % len(self.sets)
+            _, kp, vp, _ = self.sets[p]
+            n = int(self.win.plans[0].spec.chunk_video_tokens)
+            self.win.advance(kp[:, :n], vp[:, :n], stream=self.compute)
+            self.read[p].record(self.compute)
         self.win.step(q, k, v, stream=self.compute, out=o)
         computed.record(self.compute)
         with torch.cuda.stream(self.copy_back):

@@ -187,3 +187,95 @@ def test_host_step_pipeline_matches_device_step():
     pipe.synchronize()
     for r, o in zip(refs, outs):
         assert torch.equal(r, o)
+
+
+def test_host_step_pipeline_with_slides_matches_device_steps():
+    """With slide=True the pipeline slides the window by the previous step's
+    uploaded chunk before each step: outputs equal the device-side sequence
+    advance(previous chunk's video K, V) -> step, bit for bit, over enough
+    steps that the two staging sets are each reused while a slide reads the
+    other."""
+    from streaming_video_audio_b200.window import HostStepPipeline
+    spec = workloads.scaled(workloads.CHUNK_TIERED, n_heads=2)
+    n = spec.chunk_video_tokens
+    inp = workloads.draw_session(spec, 5)
+    chunks = [tuple(workloads.draw_tensor((1, spec.chunk_len, 2, 128), seed=70 + 3 * s + j) for j in range(3))
+              for s in range(6)]
+    win = StreamingWindow([spec])
+    win.load_window([inp])
+    refs = []
+    for s, (q, k, v) in enumerate(chunks):
+        if s:
+            win.advance(chunks[s - 1][1][:, :n].cuda(), chunks[s - 1][2][:, :n].cuda())
+        refs.append(win.step(q.cuda(), k.cuda(), v.cuda()).cpu().clone())
+    win2 = StreamingWindow([spec])
+    win2.load_window([inp])
+    pipe = HostStepPipeline(win2)
+    outs = [torch.empty_like(r).pin_memory() for r in refs]
+    for (q, k, v), o in zip(chunks, outs):
+        pipe.step(q.pin_memory(), k.pin_memory(), v.pin_memory(), o, slide=True)
+    pipe.synchronize()
+    win2.check_status()
+    for r, o in zip(refs, outs):
+        assert torch.equal(r, o)
+
+
+@pytest.mark.parametrize("n_frames", [3, 2])
+def test_window_slide_matches_oracle(n_frames):
+    """Streaming over successive chunks: after every slide (a1 in streaming
+    use: re-pooling at the tier boundaries, the previous chunk's clean frames
+    into the recent ring, positions of the new ring state) the step equals
+    the oracle's step on the window defined afresh one chunk later.  Chunks
+    of 2 frames make the 9- and 3-frame rings wrap inside a slide.
+
+    Window contents per ring, in age order: recent frames bit-exact, tier1
+    (pooled once) within one bf16 ulp, tier0 (re-pooled from bf16 tier1
+    frames) within the two-rounding bound 2^-9 (max|T2| + |T3|)."""
+    ft = workloads.FT
+    spec = workloads.scaled(workloads.CHUNK_TIERED, n_heads=3, prompt_len=37, chunk_video_tokens=n_frames * ft)
+    H, D, L = spec.n_heads, spec.head_dim, spec.chunk_len
+    inp = workloads.draw_session(spec, 21)
+    win = StreamingWindow([spec])
+    win.load_window([inp])
+    win.step(inp.q.cuda()[None], inp.k.cuda()[None], inp.v.cuda()[None])
+    n_slides = 13 if n_frames == 3 else 10
+    # |T2| never exceeds the largest full-resolution value that ever entered the history
+    amax = {"k": max(t.abs().max().item() for t in inp.ctx_k), "v": max(t.abs().max().item() for t in inp.ctx_v)}
+    for i in range(n_slides):
+        ck, cv = inp.k[:n_frames * ft], inp.v[:n_frames * ft]   # the finished chunk's video K / V
+        amax = {"k": max(amax["k"], ck.abs().max().item()), "v": max(amax["v"], cv.abs().max().item())}
+        q, k, v = (workloads.draw_tensor((L, H, D), seed=300 + 3 * i + j) for j in range(3))
+        win.advance(ck.cuda()[None], cv.cuda()[None])
+        win.step(q.cuda()[None], k.cuda()[None], v.cuda()[None])
+        inp = oracle.slide_window(spec, inp, ck, cv, q, k, v)
+        if i not in (0, 1, 3, n_slides - 2, n_slides - 1):
+            continue
+        torch.cuda.synchronize()
+        win.check_status()
+        rows = sample_rows(L, 24, seed=i)
+        ref_o, ref_l = oracle.session_reference(spec, inp, rows=rows)
+        o, lse = win.o.cpu(), win.lse.cpu()
+        for h in range(H):
+            mx, mean = attn_errors(o[0, rows, h], ref_o[:, h])
+            assert mx <= ATTN_MAX_ABS and mean <= ATTN_MEAN_ABS, (i, h, mx, mean)
+            # the re-pooled tier adds one rounding to its keys: twice the per-score bound
+            bound = 2.0 * (lse_bound(spec, inp, h, rows) - LSE_ABS) + LSE_ABS
+            assert np.all(np.abs(lse[0, h, rows].double().numpy() - ref_l[:, h]) <= bound), i
+        segs = {s["name"]: s for s in oracle.session_kv(spec, inp)}
+        pos = win.pos.cpu().numpy()
+        for role, r in win.rings.items():
+            order = [(win.ring_ptr[role] + j) % r["frames"] for j in range(r["frames"])]
+            off, tok = win.seg[role][0], r["tok"]
+            slots = np.concatenate([np.arange(off + s * tok, off + (s + 1) * tok) for s in order])
+            assert np.array_equal(pos[0, slots], segs[role]["pos"].astype(np.float32)), (i, role)
+            idx = torch.from_numpy(slots).cuda()
+            for buf, name in ((win.k_raw, "k"), (win.v, "v")):
+                got = buf[0][:, idx].permute(1, 0, 2).cpu()
+                ref = segs[role][name]
+                if role == "recent":
+                    assert np.array_equal(got.double().numpy(), ref), (i, role, name)
+                elif role == "tier1":
+                    assert ulp_diff_bf16(got, ref).max() <= 1, (i, role, name)
+                else:
+                    err = np.abs(got.double().numpy() - ref)
+                    assert np.all(err <= 2.0 ** -9 * (amax[name] + np.abs(ref)) + 1e-12), (i, role, name)
