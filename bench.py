@@ -265,6 +265,198 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- further rows
+ROW_DESC = {
+    "moving": "moving part of one denoising step on the tiered chunk window: queries of the 3 recent frames "
+              "(recomputed K/V written back) + the chunk attend to the whole window; 40 heads x 128",
+    "qknorm": "tiered chunk step with per-head RMSNorm of q and k fused into RoPE (keys kept before "
+              "normalisation); 40 heads x 128",
+    "window": "causal VAE decoder layer at 1/8 output resolution (96x168 tokens per frame), 512 channels as "
+              "4 heads x 128: 16x16 windows shifted by 8, 2 current + 4 ring-buffered frames",
+    "ulysses": "tiered chunk step of one session with its chunk sharded by tokens over the ranks and heads "
+               "re-partitioned by two NCCL all-to-alls (no window slide); 40 heads x 128",
+}
+
+
+def _timed(step, K, W, local, dist=None, before=None):
+    """W warm-up steps, then K steps between barriers and synchronisations;
+    step(i, marks) records `marks` around its dominant launch; `before` runs
+    on the host between the two.  Returns (total ms, mean dominant-launch ms,
+    clocks)."""
+    stream = torch.cuda.current_stream()
+    for i in range(W):
+        step(i, None)
+    torch.cuda.synchronize()
+    if before is not None:
+        before()
+    marks = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(K):
+        step(W + i, marks[i])
+    stop.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clocks = sampler.stop()
+    return start.elapsed_time(stop), float(np.mean([a.elapsed_time(b) for a, b in marks])), clocks
+
+
+def _row_line(args, world, metric, value, unit, total_ms, config, roofline, clocks, launches, scaling="weak",
+              dtype="bf16"):
+    return {"metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": scaling, "vs_baseline": None, "dtype": dtype, "data": "synthetic",
+            "config": {"workload": ROW_DESC[args.row], "row": args.row, **config},
+            "roofline": roofline, "clocks": clocks, "gpu_launches": launches, "e2e": None}
+
+
+def run_row(args, rank, world, local, device, dist):
+    """One JSON line for a row beyond the default step (rank 0 prints)."""
+    peak, _, hbm, peak_kind = peaks()
+    K, W = args.steps, args.warmup
+    from streaming_video_audio_b200.window import StreamingWindow
+    if args.row in ("moving", "qknorm"):
+        spec, seed = workloads.CHUNK_TIERED, 1000 * rank
+        inp = workloads.draw_session(spec, seed)
+        qk_norm = None
+        if args.row == "qknorm":
+            gq = 1.0 + 0.2 * workloads.draw_tensor((spec.head_dim,), seed=8).float()
+            gk = 1.0 + 0.2 * workloads.draw_tensor((spec.head_dim,), seed=9).float()
+            qk_norm = (gq, gk, 1e-6)
+        win = StreamingWindow([spec], device=device, qk_norm=qk_norm)
+        win.load_window([inp])
+        q, k, v = (getattr(inp, n).to(device)[None] for n in ("q", "k", "v"))
+        H, D = spec.n_heads, spec.head_dim
+        kv_valid = int(win.lengths.sum())
+        if args.row == "moving":
+            mov = workloads.draw_moving(spec, seed)
+            qr, kr, vr = (getattr(mov, n).to(device)[None] for n in ("recent_q", "recent_k", "recent_v"))
+            n_rec = qr.shape[1]
+
+            def step(i, marks):
+                win.step_moving(qr, kr, vr, q, k, v, marks=marks)
+
+            total, kern, clocks = _timed(step, K, W, local, dist)
+            win.check_status()
+            fl = 4.0 * (n_rec + spec.chunk_len) * kv_valid * D * H
+            ach = fl / (kern * 1e-3) / 1e12
+            roof = {"bound": "tensor", "kernel": "chunk_attention_kernel<128>", "achieved": ach, "peak": peak,
+                    "unit": "TFLOP/s", "frac": ach / peak, "peak_kind": peak_kind, "attention_ms": kern,
+                    "traffic": None}
+            value = world * fl * K / (total * 1e-3) / 1e12
+            # recent K/V append, chunk append, RoPE of chunk q, window keys, recent q, attention (+ merge)
+            launches = K * (6 + (1 if win._scratch("moving", n_rec + win.q_cap)[3] is not None else 0))
+            return _row_line(args, world, "moving-part attention TFLOP/s per denoising step", value, "TFLOP/s",
+                             total, {"q_tokens": n_rec + spec.chunk_len, "kv_tokens": kv_valid}, roof, clocks,
+                             launches)
+        n_video = spec.chunk_video_tokens
+        kc, vc = k[:, :n_video], v[:, :n_video]
+
+        def step(i, marks):
+            win.advance(kc, vc)
+            win.append_chunk(k, v)
+            win._rope(q, win.q_att.permute(0, 2, 1, 3), win.q_pos, key=False, n_valid=win.q_len)
+            if marks is not None:
+                marks[0].record()
+            win.rotate_keys()
+            if marks is not None:
+                marks[1].record()
+            win.attend()
+
+        counted = {}
+        total, kern, clocks = _timed(step, K, W, local, dist,
+                                     before=lambda: counted.update(n=launches_in_steps(win, True, K)))
+        launches = counted["n"]
+        win.check_status()
+        # algorithmic bytes of the window launch: every valid non-prompt key read
+        # (pre-norm) and written (normalised, rotated), its position, the gains
+        n_keys = kv_valid - spec.prompt_len
+        byts = n_keys * (2 * H * D * 2 + 12) + D * 4
+        ach = byts / (kern * 1e-3) / 1e9
+        roof = {"bound": "hbm", "kernel": "rope3d_kernel<128,true> (window keys)", "achieved": ach, "peak": hbm,
+                "unit": "GB/s", "frac": ach / hbm, "peak_kind": peak_kind, "kernel_ms": kern, "traffic": None,
+                "algorithmic_bytes": byts}
+        fl = 4.0 * spec.chunk_len * kv_valid * D * H
+        return _row_line(args, world, "window QK-norm + RoPE GB/s (fused launch) in the tiered chunk step", ach,
+                         "GB/s", total, {"keys": n_keys, "step_attention_tflops": world * fl * K / (total * 1e-3) / 1e12},
+                         roof, clocks, launches)
+    if args.row == "window":
+        from streaming_video_audio_b200.vae_window import RingWindowAttention
+        gh, gw, H, D = 96, 168, 4, 128
+        T = gh * gw
+        layer = RingWindowAttention((gh, gw), H, D, (32, 48, 48), shift=8, device=device)
+        frames = [tuple(workloads.draw_tensor((2 * T, H, D), seed=700 + 10 * c + j, scale=workloads.INV_SQRT2)
+                        .to(device) for j in range(3)) for c in range(2)]
+        out = torch.empty(2 * T, H, D, dtype=torch.bfloat16, device=device)
+        q_in, k_in, v_in = (torch.empty_like(out) for _ in range(3))
+        W = max(W, 6)    # the 6-frame ring is full after 3 calls; its 6 states are captured as CUDA graphs by then
+
+        def step(i, marks):
+            # each call's frames arrive in the layer's input buffers (a device copy), then
+            # the call replays from CUDA graphs
+            for dst, src in zip((q_in, k_in, v_in), frames[i % 2]):
+                dst.copy_(src)
+            layer.graphed(q_in, k_in, v_in, t0=2 * i, out=out, marks=marks)
+
+        total, kern, clocks = _timed(step, K, W, local, dist)
+        assert int(layer.status.item()) == 0
+        counts = layer.part.counts.astype(np.float64)
+        fl = float(np.sum(4.0 * (2 * counts) * (6 * counts) * D * H))
+        ach = fl / (kern * 1e-3) / 1e12
+        roof = {"bound": "tensor", "kernel": "chunk_attention_kernel<128>", "achieved": ach, "peak": peak,
+                "unit": "TFLOP/s", "frac": ach / peak, "peak_kind": peak_kind, "attention_ms": kern,
+                "traffic": None}
+        value = world * fl * K / (total * 1e-3) / 1e12
+        # per frame: gather V, gather K, RoPE of K; gather Q, RoPE of Q; attention (+ merge); scatter
+        # (plus torch's position add and the three input copies, not counted)
+        launches = K * (2 * 3 + 2 + 1 + 1 + (1 if layer.workspace is not None else 0))
+        return _row_line(args, world, "windowed attention TFLOP/s per decoder call (2 latent frames)", value,
+                         "TFLOP/s", total, {"windows": layer.part.n_windows, "tokens_per_call": 2 * T}, roof,
+                         clocks, launches)
+    if args.row == "ulysses":
+        from streaming_video_audio_b200.ulysses import UlyssesAttention
+        spec = workloads.CHUNK_TIERED
+        inp = workloads.draw_session(spec, 0)          # one session shared by all ranks
+        ua = UlyssesAttention(spec, rank, world, group=dist.group.WORLD if dist else None, device=device)
+        ua.load_window(inp)
+        lo, hi = ua.plan.tokens_of(rank)
+        q, k, v = (getattr(inp, n)[lo:hi].to(device) for n in ("q", "k", "v"))
+        out = torch.empty(hi - lo, spec.n_heads, spec.head_dim, dtype=torch.bfloat16, device=device)
+        if dist is None:
+            import torch.distributed as tdist
+            tdist.init_process_group("nccl", store=tdist.HashStore(), rank=0, world_size=1, device_id=device)
+            ua.group = tdist.group.WORLD
+
+        def step(i, marks):
+            ua.step(q, k, v, out=out, marks=marks)
+
+        total, kern, clocks = _timed(step, K, W, local, dist)
+        ua.win.check_status()
+        from streaming_video_audio_b200.window import SessionPlan
+        fl = 4.0 * spec.chunk_len * sum(SessionPlan(spec).lengths.values()) * spec.head_dim * spec.n_heads
+        agg = aggregate([total, total, kern], fl, K, 1, dist.group.WORLD if dist else None)
+        ach = fl / world / (agg["attn_ms"] * 1e-3) / 1e12
+        roof = {"bound": "tensor", "kernel": "chunk_attention_kernel<128>", "achieved": ach, "peak": peak,
+                "unit": "TFLOP/s", "frac": ach / peak, "peak_kind": peak_kind, "attention_ms": agg["attn_ms"],
+                "traffic": None}
+        launches = K * (4 + (1 if ua.win.workspace is not None else 0))
+        line = _row_line(args, world, "attention TFLOP/s of one session's streaming step (whole job)",
+                         agg["value"], "TFLOP/s", agg["total_ms"],
+                         {"heads_per_rank": ua.Hn, "tokens_per_rank": ua.S, "parallelism": f"ulysses{world}",
+                          "exchange_bytes_per_rank_per_step": int(ua.send.numel() * 2 + ua.o_recv.numel() * 2)},
+                         roof, clocks, launches, scaling="strong")
+        if dist is None:
+            import torch.distributed as tdist
+            tdist.destroy_process_group()
+        return line
+    raise ValueError(args.row)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -273,6 +465,8 @@ def main():
     ap.add_argument("--config", type=int, default=3, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--impl", default="sr", choices=["sr", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--row", default="step", choices=["step", "moving", "qknorm", "window", "ulysses"],
+                    help="step: the default streaming step; others: the further rows (one JSON line each)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -292,6 +486,15 @@ def main():
         import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+
+    if args.row != "step":
+        line = run_row(args, rank, world, local, device, dist)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        if dist:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
 
     specs, inputs, win, chunk = build_window(args.config, rank, device)
     tiered = any(s.tiers for s in specs)

@@ -61,45 +61,43 @@ struct RopeArgs {
 };
 
 // One CTA per (token, batch).  Thread t handles the 16-byte chunk
-// c = t % (D/8) of heads t/(D/8), t/(D/8) + 128/(D/8), ...  It first issues
-// the loads of all its heads (up to kIters of them in flight), then derives
-// the token's four (cos, sin) pairs -- they depend on (token, pair) only and
-// are reused for every head -- and finally rotates and stores.  The angle
-// p * theta is formed in double and reduced to [-pi, pi] in double, so its
-// error does not grow with the position's magnitude; the small remainder goes
-// through fp32 sincosf.  The rotation itself runs in fp32.
+// c = t % (D/8) of heads t/(D/8), t/(D/8) + 128/(D/8), ... (kPasses heads,
+// a compile-time count so that only the registers in use are allocated).  It
+// first issues the loads of all its heads, then derives the token's four
+// (cos, sin) pairs -- they depend on (token, pair) only and are reused for
+// every head -- and finally rotates and stores.  The angle p * theta is
+// formed in double and reduced to [-pi, pi] in double, so its error does not
+// grow with the position's magnitude; the small remainder goes through fp32
+// sincosf.  The rotation itself runs in fp32.
 // kNorm: RMSNorm of each head vector first (QK normalisation): the D/8
-// threads holding one head row reduce its sum of squares with shuffles, then
-// scale by rsqrt(mean + eps) * gamma before rotating.  Needs n_heads <=
-// kIters * (128 / (D/8)) so every thread runs the same shuffles.
-template <int D, bool kNorm>
-__global__ void __launch_bounds__(128) rope3d_kernel(const RopeArgs a, const RopeTable tab) {
+// threads holding one head row reduce its sum of squares with shuffles --
+// the reductions of all passes side by side, so their latencies overlap --
+// then scale by rsqrt(mean + eps) * gamma before rotating.  Needs n_heads <=
+// kPasses * (128 / (D/8)) so every thread runs the same shuffles.
+template <int D, bool kNorm, int kPasses>
+__global__ void __launch_bounds__(128, kPasses <= 5 ? 8 : 4) rope3d_kernel(const RopeArgs a, const RopeTable tab) {
     constexpr int kChunks = D / 8;
     constexpr int kHeadsPerPass = 128 / kChunks;
-    constexpr int kIters = 8;   // heads kept in flight per thread: 8 x 8 = 64 heads at D = 128
     const int n = blockIdx.x, b = blockIdx.y;
     if (a.n_valid && n >= a.n_valid[b]) return;   // uniform per CTA (before the barrier below)
     const int c = threadIdx.x % kChunks;
     const int hp = threadIdx.x / kChunks;
     const __nv_bfloat16 *xt = a.x + b * a.xb + n * a.xt + c * 8;
     __nv_bfloat16 *yt = a.y + b * a.yb + n * a.yt + c * 8;
-    uint4 u[kIters];
+    uint4 u[kPasses];
 #pragma unroll
-    for (int i = 0; i < kIters; ++i) {
+    for (int i = 0; i < kPasses; ++i) {
         const int h = hp + i * kHeadsPerPass;
         u[i] = h < a.n_heads ? __ldg(reinterpret_cast<const uint4 *>(xt + h * a.xh)) : make_uint4(0, 0, 0, 0);
-    }
-    float g[8];
-    if constexpr (kNorm) {
-        const float4 g0 = __ldg(reinterpret_cast<const float4 *>(a.gamma + c * 8));
-        const float4 g1 = __ldg(reinterpret_cast<const float4 *>(a.gamma + c * 8 + 4));
-        g[0] = g0.x; g[1] = g0.y; g[2] = g0.z; g[3] = g0.w;
-        g[4] = g1.x; g[5] = g1.y; g[6] = g1.z; g[7] = g1.w;
     }
     // theta per pair, staged once per CTA: indexing the parameter table with a
     // per-thread index would serialise the constant-cache reads
     __shared__ double s_theta[D / 2];
+    __shared__ __align__(16) float s_gamma[kNorm ? D : 1];   // gains, read per pass (keeps registers free)
     if (threadIdx.x < D / 2) s_theta[threadIdx.x] = tab.theta[threadIdx.x];
+    if constexpr (kNorm) {
+        if (threadIdx.x < D) s_gamma[threadIdx.x] = a.gamma[threadIdx.x];
+    }
     __syncthreads();
     float cs[4], sn[4];
     float pt = 0.f, ph = 0.f, pw = 0.f;
@@ -122,43 +120,56 @@ __global__ void __launch_bounds__(128) rope3d_kernel(const RopeArgs a, const Rop
         cs[k] = co * a.out_scale;
         sn[k] = s * a.out_scale;
     }
+    float inv[kPasses];
+    if constexpr (kNorm) {
 #pragma unroll
-    for (int i = 0; i < kIters; ++i) {
-        const int h = hp + i * kHeadsPerPass;
-        if (kNorm && i * kHeadsPerPass >= a.n_heads) break;   // uniform: no head of this pass exists
-        float f[8], r[8];
-        unpack8(u[i], f);
-        if constexpr (kNorm) {
+        for (int i = 0; i < kPasses; ++i) {
+            float f[8];
+            unpack8(u[i], f);
             float ss = 0.f;
 #pragma unroll
             for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
+            inv[i] = ss;
+        }
 #pragma unroll
-            for (int off = kChunks / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-            const float inv = rsqrtf(ss * (1.0f / D) + a.eps);
+        for (int off = kChunks / 2; off > 0; off >>= 1)
 #pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = f[e] * inv * g[e];
-            if (a.y_raw && h < a.n_heads)
+            for (int i = 0; i < kPasses; ++i) inv[i] += __shfl_xor_sync(0xffffffffu, inv[i], off);
+#pragma unroll
+        for (int i = 0; i < kPasses; ++i) inv[i] = rsqrtf(inv[i] * (1.0f / D) + a.eps);
+    }
+#pragma unroll
+    for (int i = 0; i < kPasses; ++i) {
+        const int h = hp + i * kHeadsPerPass;
+        if (h >= a.n_heads) continue;
+        float f[8], r[8];
+        unpack8(u[i], f);
+        if constexpr (kNorm) {
+            const float4 g0 = *reinterpret_cast<const float4 *>(s_gamma + c * 8);
+            const float4 g1 = *reinterpret_cast<const float4 *>(s_gamma + c * 8 + 4);
+            const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] = f[e] * inv[i] * g[e];
+            if (a.y_raw)
                 *reinterpret_cast<uint4 *>(a.y_raw + b * a.rb + n * a.rt + h * a.rh + c * 8) = pack8(f);
         }
-        if (h < a.n_heads) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                r[2 * k] = f[2 * k] * cs[k] - f[2 * k + 1] * sn[k];
-                r[2 * k + 1] = f[2 * k] * sn[k] + f[2 * k + 1] * cs[k];
-            }
-            *reinterpret_cast<uint4 *>(yt + h * a.yh) = pack8(r);
+        for (int k = 0; k < 4; ++k) {
+            r[2 * k] = f[2 * k] * cs[k] - f[2 * k + 1] * sn[k];
+            r[2 * k + 1] = f[2 * k] * sn[k] + f[2 * k + 1] * cs[k];
         }
+        *reinterpret_cast<uint4 *>(yt + h * a.yh) = pack8(r);
     }
     if constexpr (kNorm) return;   // the host guarantees n_heads fits the passes above
-    for (int h = hp + kIters * kHeadsPerPass; h < a.n_heads; h += kHeadsPerPass) {   // very many heads
-        float f[8], g[8];
+    for (int h = hp + kPasses * kHeadsPerPass; h < a.n_heads; h += kHeadsPerPass) {   // very many heads
+        float f[8], r[8];
         unpack8(__ldg(reinterpret_cast<const uint4 *>(xt + h * a.xh)), f);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            g[2 * k] = f[2 * k] * cs[k] - f[2 * k + 1] * sn[k];
-            g[2 * k + 1] = f[2 * k] * sn[k] + f[2 * k + 1] * cs[k];
+            r[2 * k] = f[2 * k] * cs[k] - f[2 * k + 1] * sn[k];
+            r[2 * k + 1] = f[2 * k] * sn[k] + f[2 * k + 1] * cs[k];
         }
-        *reinterpret_cast<uint4 *>(yt + h * a.yh) = pack8(g);
+        *reinterpret_cast<uint4 *>(yt + h * a.yh) = pack8(r);
     }
 }
 
@@ -387,7 +398,19 @@ int rope_launch(const RopeLaunch &l) {
                l.n_heads, l.out_scale, l.xb, l.xt, l.xh, l.yb, l.yt, l.yh, l.pb,
                l.gamma, l.eps, static_cast<__nv_bfloat16 *>(l.y_raw), l.rb, l.rt, l.rh};
     dim3 grid(l.n_tokens, l.n_batch);
-    rope3d_kernel<D, kNorm><<<grid, 128, 0, l.stream>>>(a, tab);
+    // passes of 128 / (D/8) heads each: instantiated for 1..8 (more heads run
+    // the extra passes in a loop, without normalisation only)
+    const int passes = (l.n_heads + 128 / (D / 8) - 1) / (128 / (D / 8));
+    switch (passes < 8 ? passes : 8) {
+        case 1: rope3d_kernel<D, kNorm, 1><<<grid, 128, 0, l.stream>>>(a, tab); break;
+        case 2: rope3d_kernel<D, kNorm, 2><<<grid, 128, 0, l.stream>>>(a, tab); break;
+        case 3: rope3d_kernel<D, kNorm, 3><<<grid, 128, 0, l.stream>>>(a, tab); break;
+        case 4: rope3d_kernel<D, kNorm, 4><<<grid, 128, 0, l.stream>>>(a, tab); break;
+        case 5: rope3d_kernel<D, kNorm, 5><<<grid, 128, 0, l.stream>>>(a, tab); break;
+        case 6: rope3d_kernel<D, kNorm, 6><<<grid, 128, 0, l.stream>>>(a, tab); break;
+        case 7: rope3d_kernel<D, kNorm, 7><<<grid, 128, 0, l.stream>>>(a, tab); break;
+        default: rope3d_kernel<D, kNorm, 8><<<grid, 128, 0, l.stream>>>(a, tab); break;
+    }
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? SR_OK : set_cuda_error("rope3d launch", e);
 }

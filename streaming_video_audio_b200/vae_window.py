@@ -31,6 +31,7 @@ import numpy as np
 import torch
 
 from . import capi
+from .window import _mark
 
 
 class WindowPartition:
@@ -102,7 +103,14 @@ class RingWindowAttention:
             self.kv_len_phase.append(torch.from_numpy(lens).to(self.device))
         ws = capi.sr_chunk_attention_workspace_bytes(W, H, D, self.q_cap)
         self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, **kw) if ws else None
+        # positions of the current frames: (f, row, col) + t0 on the t axis,
+        # formed on the device so that a call never waits for the host
+        self.pos_base = self.frame_positions(0)
+        self.t_axis = torch.tensor([1.0, 0.0, 0.0], **kw)
+        self.t0_dev = torch.zeros(1, **kw)
+        self.pos_cur = torch.zeros_like(self.pos_base)
         self.calls = 0
+        self.graphs = {}
 
     def frame_positions(self, t0: int) -> torch.Tensor:
         """(t, h, w) of the current frames' tokens, t absolute."""
@@ -111,35 +119,88 @@ class RingWindowAttention:
         pos = [np.stack([np.full(gh * gw, t0 + f), r, c], axis=1) for f in range(self.fpc)]
         return torch.from_numpy(np.concatenate(pos).astype(np.float32)).to(self.device)
 
-    def __call__(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, t0: int,
-                 out: torch.Tensor = None, stream=None) -> torch.Tensor:
-        """q, k, v: the current frames' tokens [frames_per_call * gh * gw, H, D]
-        (token-major, before RoPE); t0: absolute latent index of the first
-        current frame.  Returns o of the same shape."""
-        n_tok = self.fpc * self.part.gh * self.part.gw
-        assert q.shape == (n_tok, self.H, self.D) and k.shape == q.shape and v.shape == q.shape
-        if out is None:
-            out = torch.zeros_like(q)
-        W, H, D, S = self.part.n_windows, self.H, self.D, self.slot_cap
-        pos = self.frame_positions(t0)
-        slot0 = (self.calls * self.fpc) % self.slots
+    def _state(self):
+        """(first ring slot of this call, valid-length phase) from the call count."""
+        return (self.calls * self.fpc) % self.slots, min(self.calls, len(self.kv_len_phase) - 1)
+
+    def _prepare(self, q, k, v, slot0: int, stream=None) -> None:
+        """Positions, cache write of the current frames' K (RoPE) and V, partition
+        and RoPE of the queries."""
+        S = self.slot_cap
+        torch.addcmul(self.pos_base, self.t_axis, self.t0_dev, out=self.pos_cur)
         for f in range(self.fpc):
             sl = (slot0 + f) % self.slots
             ring_k = self.k_ring[:, :, sl * S:(sl + 1) * S]
             ring_v = self.v_ring[:, :, sl * S:(sl + 1) * S]
             # V straight into its ring slot; K through a staging buffer for its one-time RoPE
             self._gather(ring_v.permute(0, 2, 1, 3), v, self.idx_kv[f], stream=stream)
-            self._gather(self.k_tmp, k, self.idx_kv[f], pos=pos, pos_out=self.pos_k, stream=stream)
+            self._gather(self.k_tmp, k, self.idx_kv[f], pos=self.pos_cur, pos_out=self.pos_k, stream=stream)
             capi.sr_rope3d_apply(self.k_tmp, ring_k.permute(0, 2, 1, 3), self.pos_k, self.split, self.base,
                                  stream=stream)
-        self._gather(self.q_tmp, q, self.idx_q, pos=pos, pos_out=self.pos_q, stream=stream)
+        self._gather(self.q_tmp, q, self.idx_q, pos=self.pos_cur, pos_out=self.pos_q, stream=stream)
         capi.sr_rope3d_apply(self.q_tmp, self.q_att.permute(0, 2, 1, 3), self.pos_q, self.split, self.base,
                              stream=stream)
-        phase = min(self.calls, len(self.kv_len_phase) - 1)
+
+    def _attend(self, phase: int, stream=None) -> None:
+        S = self.slot_cap
         capi.sr_chunk_attention_fwd(self.q_att, self.k_ring, self.v_ring, self.o_win, self.lse,
-                                    [S] * self.slots, self.kv_len_phase[phase], self.q_len, 1.0 / math.sqrt(D),
-                                    self.status, workspace=self.workspace, stream=stream)
+                                    [S] * self.slots, self.kv_len_phase[phase], self.q_len,
+                                    1.0 / math.sqrt(self.D), self.status, workspace=self.workspace, stream=stream)
+
+    def _merge(self, out, stream=None) -> None:
         capi.sr_scatter_tokens(out, self.o_win, self.idx_q, stream=stream)
+
+    def __call__(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, t0: int,
+                 out: torch.Tensor = None, stream=None, marks=None) -> torch.Tensor:
+        """q, k, v: the current frames' tokens [frames_per_call * gh * gw, H, D]
+        (token-major, before RoPE); t0: absolute latent index of the first
+        current frame.  Returns o of the same shape.  `marks`: optional pair
+        of CUDA events recorded around the attention launch."""
+        n_tok = self.fpc * self.part.gh * self.part.gw
+        assert q.shape == (n_tok, self.H, self.D) and k.shape == q.shape and v.shape == q.shape
+        if out is None:
+            out = torch.zeros_like(q)
+        slot0, phase = self._state()
+        self.t0_dev.fill_(float(t0))
+        self._prepare(q, k, v, slot0, stream)
+        _mark(marks, 0, stream)
+        self._attend(phase, stream)
+        _mark(marks, 1, stream)
+        self._merge(out, stream)
+        self.calls += 1
+        return out
+
+    def graphed(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, t0: int, out: torch.Tensor,
+                marks=None) -> torch.Tensor:
+        """The same call replayed from CUDA graphs (no per-launch host work).
+
+        q, k, v and out must be the same tensors (addresses) on every call.
+        Each ring state (first slot, valid-length phase) -- five in all for
+        the default 2 + 4 frames -- is captured the first time it occurs,
+        after that call has run eagerly; a call then costs three graph launches
+        (prepare, attention, merge) on the current stream, with `marks`
+        recorded around the attention graph."""
+        slot0, phase = self._state()
+        key = (slot0, phase)
+        if key not in self.graphs:
+            self(q, k, v, t0, out=out, marks=marks)
+            torch.cuda.synchronize()
+            gs = [torch.cuda.CUDAGraph() for _ in range(3)]
+            with torch.cuda.graph(gs[0]):
+                self._prepare(q, k, v, slot0)
+            with torch.cuda.graph(gs[1]):
+                self._attend(phase)
+            with torch.cuda.graph(gs[2]):
+                self._merge(out)
+            self.graphs[key] = gs
+            return out
+        gs = self.graphs[key]
+        self.t0_dev.fill_(float(t0))
+        gs[0].replay()
+        _mark(marks, 0, None)
+        gs[1].replay()
+        _mark(marks, 1, None)
+        gs[2].replay()
         self.calls += 1
         return out
 

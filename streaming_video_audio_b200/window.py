@@ -45,6 +45,12 @@ from . import capi
 TILE = capi.SR_TILE
 
 
+def _mark(marks, i: int, stream) -> None:
+    """Record event i of an optional (before, after) pair on `stream`."""
+    if marks is not None:
+        marks[i].record(stream if stream is not None else torch.cuda.current_stream())
+
+
 def _ceil_div(a: int, b: int) -> int:
     return -(-a // b)
 
@@ -267,21 +273,24 @@ class StreamingWindow:
             capi.sr_qknorm_rope3d_apply(x, y, gk if key else gq, eps, pos, self.split, self.base, n_valid=n_valid,
                                         stream=stream)
 
-    def attend(self, stream=None, out: torch.Tensor = None) -> torch.Tensor:
+    def attend(self, stream=None, out: torch.Tensor = None, marks=None) -> torch.Tensor:
         """a4: fused chunk attention -> o [B, q_cap, H, D] (and lse); `out`
-        optionally replaces the window's own output buffer."""
+        optionally replaces the window's own output buffer; `marks`, a pair
+        of CUDA events, is recorded around the launch (for timing)."""
         o = self.o if out is None else out
+        _mark(marks, 0, stream)
         capi.sr_chunk_attention_fwd(self.q_att, self.k_att, self.v, o, self.lse, self.caps, self.kv_len,
                                     self.q_len, self.scale, self.status, workspace=self.workspace, stream=stream)
+        _mark(marks, 1, stream)
         return o
 
     def step(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream=None,
-             out: torch.Tensor = None) -> torch.Tensor:
+             out: torch.Tensor = None, marks=None) -> torch.Tensor:
         """One streaming attention step: a2 -> a3 -> a4 (device tensors
         [B, q_cap, H, D], token-major, pre-RoPE)."""
         self.append_chunk(k, v, stream)
         self.rotate(q, stream)
-        return self.attend(stream, out=out)
+        return self.attend(stream, out=out, marks=marks)
 
     def step_from_host(self, q_host: torch.Tensor, k_host: torch.Tensor, v_host: torch.Tensor,
                        o_host: torch.Tensor, staging=None, stream=None) -> torch.Tensor:
@@ -315,40 +324,52 @@ class StreamingWindow:
             out[b, :x.shape[0]] = x
         return out
 
+    def _scratch(self, key: str, n_q: int):
+        """Per-shape buffers of the prefix / moving attention, allocated once:
+        q_att [B, H, n_q, D], o [B, n_q, H, D], lse, the split workspace."""
+        cache = self.__dict__.setdefault("_scratch_bufs", {})
+        if (key, n_q) not in cache:
+            B, H, D, dev = self.B, self.H, self.D, self.device
+            ws_bytes = capi.sr_chunk_attention_workspace_bytes(B, H, D, n_q)
+            cache[(key, n_q)] = (torch.zeros(B, H, n_q, D, dtype=torch.bfloat16, device=dev),
+                                 torch.zeros(B, n_q, H, D, dtype=torch.bfloat16, device=dev),
+                                 torch.zeros(B, H, n_q, dtype=torch.float32, device=dev),
+                                 torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev) if ws_bytes else None)
+        return cache[(key, n_q)]
+
     def attend_prefix(self, q_prefix: torch.Tensor, stream=None) -> torch.Tensor:
         """Prefix-self attention: queries of the prefix tokens (prompt, then
         sink), token-major [B, prefix_cap, H, D] before RoPE, over the prefix
         keys only.  Returns o [B, prefix_cap, H, D] (rows past a session's
-        prefix length are left alone)."""
+        prefix length are left alone; the buffer is reused by later calls)."""
         B, n_pre, H, D = q_prefix.shape
-        pos = torch.from_numpy(self.prefix_positions()).to(self.device)
+        if not hasattr(self, "_prefix_meta"):
+            pos = torch.from_numpy(self.prefix_positions()).to(self.device)
+            lens = torch.tensor([p.lengths["prompt"] + p.lengths.get("sink", 0) for p in self.plans],
+                                dtype=torch.int32, device=self.device)
+            kv_len = self.kv_len.clone()
+            for si, name in enumerate(self.segments):
+                if name not in ("prompt", "sink"):
+                    kv_len[:, si] = 0
+            self._prefix_meta = (pos, lens, kv_len)
+        pos, lens, kv_len = self._prefix_meta
         assert n_pre == pos.shape[1], "q_prefix must cover prompt + sink tokens"
-        lens = torch.tensor([p.lengths["prompt"] + p.lengths.get("sink", 0) for p in self.plans],
-                            dtype=torch.int32, device=self.device)
-        q_att = torch.empty(B, H, n_pre, D, dtype=torch.bfloat16, device=self.device)
-        o = torch.zeros(B, n_pre, H, D, dtype=torch.bfloat16, device=self.device)
-        lse = torch.empty(B, H, n_pre, dtype=torch.float32, device=self.device)
+        q_att, o, lse, ws = self._scratch("prefix", n_pre)
         self.rotate_keys(stream)
         self._rope(q_prefix, q_att.permute(0, 2, 1, 3), pos, key=False, n_valid=lens, stream=stream)
-        kv_len = self.kv_len.clone()
-        for si, name in enumerate(self.segments):
-            if name not in ("prompt", "sink"):
-                kv_len[:, si] = 0
-        ws_bytes = capi.sr_chunk_attention_workspace_bytes(B, H, D, n_pre)
-        ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=self.device) if ws_bytes else None
         capi.sr_chunk_attention_fwd(q_att, self.k_att, self.v, o, lse, self.caps, kv_len, lens, self.scale,
                                     self.status, workspace=ws, stream=stream)
         self.prefix_lse = lse
         return o
 
     def step_moving(self, q_recent: torch.Tensor, k_recent: torch.Tensor, v_recent: torch.Tensor,
-                    q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream=None) -> torch.Tensor:
+                    q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream=None, marks=None) -> torch.Tensor:
         """The moving part of one denoising step: the recent frames' recomputed
         K (before RoPE) and V replace the recent segment, the chunk's K and V
         the chunk segment, and the queries of the recent frames followed by
         the chunk attend to the whole window.  Recent tensors [B, n_recent,
         H, D] (every session the same n_recent), chunk tensors as in step().
-        Returns o [B, n_recent + q_cap, H, D]."""
+        Returns o [B, n_recent + q_cap, H, D] (a buffer reused by later calls)."""
         B, n_rec, H, D = q_recent.shape
         off_r, _ = self.seg["recent"]
         if any(p.lengths["recent"] != n_rec for p in self.plans):
@@ -369,22 +390,23 @@ class StreamingWindow:
             capi.sr_kv_append(self.k_raw, self.v, None, off_r + slot * ft, k_recent[:, rows], v_recent[:, rows],
                               None, stream=stream)
         self.append_chunk(k, v, stream)
-        self.rotate(q, stream)   # window keys + chunk queries (the latter reused below)
         n_mov = n_rec + self.q_cap
-        q_att = torch.empty(B, H, n_mov, D, dtype=torch.bfloat16, device=self.device)
-        q_att[:, :, n_rec:].copy_(self.q_att)
+        q_att, o, lse, ws = self._scratch("moving", n_mov)
+        # chunk queries straight into their rows of the moving query buffer
+        self._rope(q, q_att[:, :, n_rec:].permute(0, 2, 1, 3), self.q_pos, key=False, n_valid=self.q_len,
+                   stream=stream)
+        self.rotate_keys(stream)
         if len(runs) == 1:
             pos_r = self.pos[:, off_r:off_r + n_rec]
         else:   # a wrapped ring holds whole frames only
             pos_r = torch.cat([self.pos[:, off_r + slot * ft:off_r + (slot + m) * ft] for slot, _, m in runs], dim=1)
         self._rope(q_recent, q_att[:, :, :n_rec].permute(0, 2, 1, 3), pos_r, key=False, stream=stream)
-        o = torch.zeros(B, n_mov, H, D, dtype=torch.bfloat16, device=self.device)
-        lse = torch.empty(B, H, n_mov, dtype=torch.float32, device=self.device)
-        q_len = self.q_len + n_rec
-        ws_bytes = capi.sr_chunk_attention_workspace_bytes(B, H, D, n_mov)
-        ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=self.device) if ws_bytes else None
-        capi.sr_chunk_attention_fwd(q_att, self.k_att, self.v, o, lse, self.caps, self.kv_len, q_len, self.scale,
-                                    self.status, workspace=ws, stream=stream)
+        if not hasattr(self, "_moving_q_len") or self._moving_q_len[0] != n_rec:
+            self._moving_q_len = (n_rec, self.q_len + n_rec)
+        _mark(marks, 0, stream)
+        capi.sr_chunk_attention_fwd(q_att, self.k_att, self.v, o, lse, self.caps, self.kv_len,
+                                    self._moving_q_len[1], self.scale, self.status, workspace=ws, stream=stream)
+        _mark(marks, 1, stream)
         self.moving_lse = lse
         return o
 

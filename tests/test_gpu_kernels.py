@@ -318,6 +318,27 @@ def test_ring_window_attention_matches_oracle(D, split, shift):
         assert mx <= ATTN_MAX_ABS and mean <= ATTN_MEAN_ABS, (c, mx, mean)
 
 
+def test_ring_window_attention_graph_replay_equals_eager_calls():
+    """Eight calls (every ring state twice) replayed from CUDA graphs give the
+    eager calls' outputs bit for bit; inputs change in place between calls."""
+    from streaming_video_audio_b200.vae_window import RingWindowAttention
+    gh, gw, H, D, T = 20, 36, 2, 128, 20 * 36
+    frames = [tuple(workloads.draw_tensor((2 * T, H, D), seed=130 + 3 * c + j) for j in range(3)) for c in range(8)]
+    eager = RingWindowAttention((gh, gw), H, D, (32, 48, 48), shift=8)
+    ref = [eager(*(t.cuda() for t in fr), t0=5 + 2 * c).cpu() for c, fr in enumerate(frames)]
+    layer = RingWindowAttention((gh, gw), H, D, (32, 48, 48), shift=8)
+    q, k, v = (torch.zeros(2 * T, H, D, dtype=torch.bfloat16, device=DEV) for _ in range(3))
+    out = torch.zeros(2 * T, H, D, dtype=torch.bfloat16, device=DEV)
+    for c, fr in enumerate(frames):
+        for dst, src in zip((q, k, v), fr):
+            dst.copy_(src)
+        layer.graphed(q, k, v, t0=5 + 2 * c, out=out)
+        torch.cuda.synchronize()
+        assert int(layer.status.item()) == 0
+        assert torch.equal(out.cpu(), ref[c]), c
+    assert len(layer.graphs) == 5     # (first slot, phase): (0,0) (2,1) (4,2) (0,2) (2,2)
+
+
 def test_ring_window_attention_is_causal_and_clock_invariant():
     """Changing a later call's frames leaves earlier outputs bit-identical, and
     starting the stream clock elsewhere changes nothing but rounding."""
