@@ -412,9 +412,9 @@ def run_row(args, rank, world, local, device, dist):
                 "unit": "TFLOP/s", "frac": ach / peak, "peak_kind": peak_kind, "attention_ms": kern,
                 "traffic": None}
         value = world * fl * K / (total * 1e-3) / 1e12
-        # per frame: gather V, gather K, RoPE of K; gather Q, RoPE of Q; attention (+ merge); scatter
-        # (plus torch's position add and the three input copies, not counted)
-        launches = K * (2 * 3 + 2 + 1 + 1 + (1 if layer.workspace is not None else 0))
+        # per frame: gather of V, gather + RoPE of K; gather + RoPE of Q; attention (+ merge);
+        # scatter (plus torch's position add and the three input copies, not counted)
+        launches = K * (2 * 2 + 1 + 1 + 1 + (1 if layer.workspace is not None else 0))
         return _row_line(args, world, "windowed attention TFLOP/s per decoder call (2 latent frames)", value,
                          "TFLOP/s", total, {"windows": layer.part.n_windows, "tokens_per_call": 2 * T}, roof,
                          clocks, launches)

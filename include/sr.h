@@ -212,6 +212,26 @@ int sr_scatter_tokens(void *dst, const void *src, const int32_t *idx, int32_t n_
                       int32_t n_heads, int32_t head_dim, int64_t dst_token_stride, int64_t dst_head_stride,
                       int64_t src_batch_stride, int64_t src_slot_stride, int64_t src_head_stride, void *stream);
 
+/* Gather with RoPE: the gather above with every copied row rotated by its
+ * source token's position on the way, i.e. the positional encoding and the
+ * cache write of the windowed KV ring in one pass.
+ *
+ * Defined by: "StreamRender-H3" (molayo1419.me), causal VAE section: the
+ * position encoding and the cache write happen once, when a frame enters the
+ * ring, and partition is an index gather; the rotation is the one of
+ * sr_rope3d_apply (3-D RoPE, interleaved pairs in t/h/w sub-blocks).
+ *
+ *   dst[b][s][h][:] = idx[b][s] >= 0 ? R(src_pos[idx[b][s]]) src[idx[b][s]][h][:] * out_scale : 0
+ * Strides as for sr_gather_tokens; src_pos: fp32 [tokens][3] (t, h, w),
+ * required.  cfg as for sr_rope3d_apply (sub-blocks multiples of 8 summing
+ * to head_dim).  head_dim in {64, 128}.  Returns SR_ERR_INVALID_ARG (nothing
+ * launched) for bad sizes, strides, alignment or a missing src_pos.
+ */
+int sr_gather_rope3d_tokens(void *dst, const void *src, const int32_t *idx, const float *src_pos, int32_t n_batch,
+                            int32_t n_slots, int32_t n_heads, int32_t head_dim, sr_rope_cfg cfg, float out_scale,
+                            int64_t src_token_stride, int64_t src_head_stride, int64_t dst_batch_stride,
+                            int64_t dst_slot_stride, int64_t dst_head_stride, void *stream);
+
 /* ------------------------------------------------------------------------ */
 /* Fused chunk attention over [prompt | context | chunk] KV segments.
  *

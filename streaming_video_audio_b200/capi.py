@@ -60,6 +60,8 @@ _SIGS = {
     "sr_gather_tokens": ([_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i64, _i64, _i64, _i64, _i64, _vp, _vp, _i64, _vp],
                          ctypes.c_int),
     "sr_scatter_tokens": ([_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i64, _i64, _i64, _i64, _i64, _vp], ctypes.c_int),
+    "sr_gather_rope3d_tokens": ([_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, sr_rope_cfg, _f32,
+                                 _i64, _i64, _i64, _i64, _i64, _vp], ctypes.c_int),
     "sr_history_compress": ([_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, sr_pool_cfg,
                              _i64, _i64, _i64, _i64, _i64, _i64, _i64, _i64, _vp, _vp, _i64, _vp, _vp],
                             ctypes.c_int),
@@ -201,6 +203,27 @@ def sr_gather_tokens(dst: torch.Tensor, src: torch.Tensor, idx: torch.Tensor, sr
     _check("sr_gather_tokens", load().sr_gather_tokens(
         _ptr(dst), _ptr(src), _ptr(idx), B, S, H, D, src.stride(0), src.stride(1), dst.stride(0), dst.stride(1),
         dst.stride(2), _ptr(src_pos), _ptr(dst_pos), pb, _stream(stream)))
+
+
+def sr_gather_rope3d_tokens(dst: torch.Tensor, src: torch.Tensor, idx: torch.Tensor, src_pos: torch.Tensor,
+                            split: Sequence[int], base: float = 10000.0, out_scale: float = 1.0, stream=None) -> None:
+    """As sr_gather_tokens, every copied row rotated by the 3-D RoPE of its
+    source token's position src_pos [T, 3] (fp32, contiguous)."""
+    for t, n in ((dst, "dst"), (src, "src")):
+        _cuda(t, torch.bfloat16, n)
+    _cuda(idx, torch.int32, "idx")
+    _cuda(src_pos, torch.float32, "src_pos")
+    B, S, H, D = dst.shape
+    if src.dim() != 3 or src.shape[1:] != (H, D) or src.stride(2) != 1 or dst.stride(3) != 1:
+        raise ValueError("src must be [T, H, D] and dst [B, S, H, D] with contiguous D")
+    if tuple(idx.shape) != (B, S) or not idx.is_contiguous():
+        raise ValueError("idx must be contiguous int32 [B, S]")
+    if src_pos is None or src_pos.shape != (src.shape[0], 3) or not src_pos.is_contiguous():
+        raise ValueError("src_pos must be contiguous fp32 [T, 3]")
+    cfg = sr_rope_cfg(float(base), int(split[0]), int(split[1]), int(split[2]))
+    _check("sr_gather_rope3d_tokens", load().sr_gather_rope3d_tokens(
+        _ptr(dst), _ptr(src), _ptr(idx), _ptr(src_pos), B, S, H, D, cfg, float(out_scale), src.stride(0),
+        src.stride(1), dst.stride(0), dst.stride(1), dst.stride(2), _stream(stream)))
 
 
 def sr_scatter_tokens(dst: torch.Tensor, src: torch.Tensor, idx: torch.Tensor, stream=None) -> None:

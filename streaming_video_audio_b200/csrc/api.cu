@@ -208,6 +208,33 @@ int sr_scatter_tokens(void *dst, const void *src, const int32_t *idx, int32_t n_
     return launch_gather(l);
 }
 
+int sr_gather_rope3d_tokens(void *dst, const void *src, const int32_t *idx, const float *src_pos, int32_t n_batch,
+                            int32_t n_slots, int32_t n_heads, int32_t head_dim, sr_rope_cfg cfg, float out_scale,
+                            int64_t src_token_stride, int64_t src_head_stride, int64_t dst_batch_stride,
+                            int64_t dst_slot_stride, int64_t dst_head_stride, void *stream) {
+    g_last_error[0] = 0;
+    GatherLaunch l{};
+    int rc = gather_common("gather_rope3d_tokens", dst, src, idx, n_batch, n_slots, n_heads, head_dim,
+                           src_token_stride, src_head_stride, dst_batch_stride, dst_slot_stride, dst_head_stride, l);
+    if (rc != SR_OK) return rc < 0 ? SR_OK : rc;
+    if (cfg.d_t < 0 || cfg.d_h < 0 || cfg.d_w < 0 || cfg.d_t % 8 || cfg.d_h % 8 || cfg.d_w % 8 ||
+        cfg.d_t + cfg.d_h + cfg.d_w != head_dim)
+        return set_error(SR_ERR_INVALID_ARG, "gather_rope3d_tokens: sub-blocks %d/%d/%d must be multiples of 8 "
+                         "summing to %d", cfg.d_t, cfg.d_h, cfg.d_w, head_dim);
+    if (!(cfg.base > 0.f)) return set_error(SR_ERR_INVALID_ARG, "gather_rope3d_tokens: base must be positive");
+    if (!src_pos || (reinterpret_cast<uintptr_t>(src_pos) & 3u))
+        return set_error(SR_ERR_INVALID_ARG, "gather_rope3d_tokens: src_pos (4-byte aligned) is required");
+    l.dst = dst;
+    l.src = src;
+    l.src_pos = src_pos;
+    l.scatter = false;
+    l.rope = true;
+    l.cfg = cfg;
+    l.out_scale = out_scale;
+    l.stream = static_cast<cudaStream_t>(stream);
+    return launch_gather(l);
+}
+
 int sr_history_compress(const void *k_in, const void *v_in, void *k_out, void *v_out, int32_t n_batch,
                         int32_t n_frames, int32_t n_heads, int32_t head_dim, sr_pool_cfg cfg, int64_t in_batch_stride,
                         int64_t in_frame_stride, int64_t in_token_stride, int64_t in_head_stride,

@@ -75,6 +75,9 @@ struct GatherLaunch {
     int32_t n_batch, n_slots, n_heads, head_dim;
     int64_t src_t, src_h, dst_b, dst_s, dst_h, pos_b;
     bool scatter;
+    bool rope;           // gather only: rotate each row by src_pos[idx] on the way
+    sr_rope_cfg cfg;
+    float out_scale;
     cudaStream_t stream;
 };
 int launch_gather(const GatherLaunch &l);

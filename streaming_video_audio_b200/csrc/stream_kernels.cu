@@ -60,6 +60,63 @@ struct RopeArgs {
     int64_t rb, rt, rh;
 };
 
+// (cos, sin) * scale of one pair: the angle p * theta is formed in double and
+// reduced to [-pi, pi] in double, so its error does not grow with the
+// position's magnitude; the small remainder goes through fp32 sincosf.
+__device__ __forceinline__ float2 pair_rotation(const RopeTable &tab, int pair, float pt, float ph, float pw,
+                                                float scale) {
+    constexpr double kTwoPi = 6.283185307179586476925286766559;
+    constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
+    const double pa = pair < tab.pairs_t ? pt : (pair < tab.pairs_th ? ph : pw);
+    const double phi = pa * tab.theta[pair];
+    const double r = fma(-rint(phi * kInvTwoPi), kTwoPi, phi);
+    float s, co;
+    sincosf(static_cast<float>(r), &s, &co);
+    return make_float2(co * scale, s * scale);
+}
+
+// The token's four (cos, sin) pairs of chunk c (pairs 4c .. 4c+3), computed
+// as pair_rotation does; s_theta: the per-pair theta in shared memory.
+__device__ __forceinline__ void token_rotation(const double *s_theta, const RopeTable &tab, int c, float pt,
+                                               float ph, float pw, float scale, float (&cs)[4], float (&sn)[4]) {
+    constexpr double kTwoPi = 6.283185307179586476925286766559;
+    constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int pair = c * 4 + k;
+        const double pa = pair < tab.pairs_t ? pt : (pair < tab.pairs_th ? ph : pw);
+        const double phi = pa * s_theta[pair];
+        const double r = fma(-rint(phi * kInvTwoPi), kTwoPi, phi);
+        float s, co;
+        sincosf(static_cast<float>(r), &s, &co);
+        cs[k] = co * scale;
+        sn[k] = s * scale;
+    }
+}
+
+__device__ __forceinline__ uint4 rotate8(const uint4 &u, const float (&cs)[4], const float (&sn)[4]) {
+    float f[8], r[8];
+    unpack8(u, f);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        r[2 * k] = f[2 * k] * cs[k] - f[2 * k + 1] * sn[k];
+        r[2 * k + 1] = f[2 * k] * sn[k] + f[2 * k + 1] * cs[k];
+    }
+    return pack8(r);
+}
+
+RopeTable make_rope_table(const sr_rope_cfg &cfg) {
+    RopeTable tab{};
+    const int widths[3] = {cfg.d_t, cfg.d_h, cfg.d_w};
+    int pair = 0;
+    for (int ax = 0; ax < 3; ++ax)
+        for (int j = 0; j < widths[ax] / 2; ++j, ++pair)
+            tab.theta[pair] = std::pow(static_cast<double>(cfg.base), -2.0 * static_cast<double>(j) / widths[ax]);
+    tab.pairs_t = cfg.d_t / 2;
+    tab.pairs_th = (cfg.d_t + cfg.d_h) / 2;
+    return tab;
+}
+
 // One CTA per (token, batch).  Thread t handles the 16-byte chunk
 // c = t % (D/8) of heads t/(D/8), t/(D/8) + 128/(D/8), ... (kPasses heads,
 // a compile-time count so that only the registers in use are allocated).  It
@@ -90,35 +147,31 @@ __global__ void __launch_bounds__(128, kPasses <= 5 ? 8 : 4) rope3d_kernel(const
         const int h = hp + i * kHeadsPerPass;
         u[i] = h < a.n_heads ? __ldg(reinterpret_cast<const uint4 *>(xt + h * a.xh)) : make_uint4(0, 0, 0, 0);
     }
-    // theta per pair, staged once per CTA: indexing the parameter table with a
-    // per-thread index would serialise the constant-cache reads
-    __shared__ double s_theta[D / 2];
+    // The token's D/2 (cos, sin) pairs, one per thread of the first D/2, shared
+    // through shared memory: every head-row group of the CTA needs the same
+    // pairs of its chunk, so each is evaluated once per token.
+    __shared__ __align__(16) float2 s_rot[D / 2];
     __shared__ __align__(16) float s_gamma[kNorm ? D : 1];   // gains, read per pass (keeps registers free)
-    if (threadIdx.x < D / 2) s_theta[threadIdx.x] = tab.theta[threadIdx.x];
+    if (threadIdx.x < D / 2) {
+        float pt = 0.f, ph = 0.f, pw = 0.f;
+        if (a.pos) {
+            const float *pp = a.pos + b * a.pb + 3 * static_cast<int64_t>(n);
+            pt = pp[0];
+            ph = pp[1];
+            pw = pp[2];
+        }
+        s_rot[threadIdx.x] = pair_rotation(tab, threadIdx.x, pt, ph, pw, a.out_scale);
+    }
     if constexpr (kNorm) {
         if (threadIdx.x < D) s_gamma[threadIdx.x] = a.gamma[threadIdx.x];
     }
     __syncthreads();
     float cs[4], sn[4];
-    float pt = 0.f, ph = 0.f, pw = 0.f;
-    if (a.pos) {
-        const float *pp = a.pos + b * a.pb + 3 * static_cast<int64_t>(n);
-        pt = pp[0];
-        ph = pp[1];
-        pw = pp[2];
-    }
-    constexpr double kTwoPi = 6.283185307179586476925286766559;
-    constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int pair = c * 4 + k;
-        const double pa = pair < tab.pairs_t ? pt : (pair < tab.pairs_th ? ph : pw);
-        const double phi = pa * s_theta[pair];
-        const double r = fma(-rint(phi * kInvTwoPi), kTwoPi, phi);
-        float s, co;
-        sincosf(static_cast<float>(r), &s, &co);
-        cs[k] = co * a.out_scale;
-        sn[k] = s * a.out_scale;
+    {
+        const float4 r01 = *reinterpret_cast<const float4 *>(s_rot + c * 4);
+        const float4 r23 = *reinterpret_cast<const float4 *>(s_rot + c * 4 + 2);
+        cs[0] = r01.x; sn[0] = r01.y; cs[1] = r01.z; sn[1] = r01.w;
+        cs[2] = r23.x; sn[2] = r23.y; cs[3] = r23.z; sn[3] = r23.w;
     }
     float inv[kPasses];
     if constexpr (kNorm) {
@@ -161,16 +214,9 @@ __global__ void __launch_bounds__(128, kPasses <= 5 ? 8 : 4) rope3d_kernel(const
         *reinterpret_cast<uint4 *>(yt + h * a.yh) = pack8(r);
     }
     if constexpr (kNorm) return;   // the host guarantees n_heads fits the passes above
-    for (int h = hp + kPasses * kHeadsPerPass; h < a.n_heads; h += kHeadsPerPass) {   // very many heads
-        float f[8], r[8];
-        unpack8(__ldg(reinterpret_cast<const uint4 *>(xt + h * a.xh)), f);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            r[2 * k] = f[2 * k] * cs[k] - f[2 * k + 1] * sn[k];
-            r[2 * k + 1] = f[2 * k] * sn[k] + f[2 * k + 1] * cs[k];
-        }
-        *reinterpret_cast<uint4 *>(yt + h * a.yh) = pack8(r);
-    }
+    for (int h = hp + kPasses * kHeadsPerPass; h < a.n_heads; h += kHeadsPerPass)   // very many heads
+        *reinterpret_cast<uint4 *>(yt + h * a.yh) =
+            rotate8(__ldg(reinterpret_cast<const uint4 *>(xt + h * a.xh)), cs, sn);
 }
 
 // ============================================================== pooling
@@ -319,38 +365,70 @@ struct GatherArgs {
     void *__restrict__ dst;
     const void *__restrict__ src;
     const int32_t *__restrict__ idx;   // [n_batch][n_slots]: source token, or < 0
-    const float *__restrict__ src_pos; // gather only: [tokens][3] or null
+    const float *__restrict__ src_pos; // gather only: [tokens][3] or null (required for RoPE)
     float *__restrict__ dst_pos;       // gather only: [n_batch][n_slots][3] or null
     int32_t n_slots, n_heads;
     int64_t src_t, src_h, dst_b, dst_s, dst_h, pos_b;
-    int64_t total;                     // threads per batch entry
+    int64_t total;                     // threads per batch entry: slots x D/8
+    float out_scale;                   // RoPE gather only
 };
 
-// dst[b][s][h][:] = idx >= 0 ? src[idx][h][:] : 0   (and the positions likewise)
-template <int D>
-__global__ void __launch_bounds__(256) gather_kernel(const GatherArgs a) {
+constexpr int kGatherHeads = 8;   // head rows a thread keeps in flight
+
+// One thread per (batch, slot, 16-byte chunk), chunk fastest: half a warp
+// covers one 256-byte head row of a token.  The thread walks the token's
+// heads 8 at a time with all 8 loads in flight.
+// Gather: dst[b][s][h][:] = idx >= 0 ? src[idx][h][:] : 0 (positions likewise);
+// kRope: the row is rotated by the position src_pos[idx] on the way (the
+// cache write and the RoPE in one pass), the token's (cos, sin) pairs
+// computed once for all its heads.
+template <int D, bool kRope>
+__global__ void __launch_bounds__(256) gather_kernel(const GatherArgs a, const RopeTable tab) {
     constexpr int kChunks = D / 8;
+    __shared__ double s_theta[kRope ? D / 2 : 1];
+    if constexpr (kRope) {
+        if (threadIdx.x < D / 2) s_theta[threadIdx.x] = tab.theta[threadIdx.x];
+        __syncthreads();
+    }
     const uint32_t i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= static_cast<uint32_t>(a.total)) return;
     const int b = blockIdx.y;
     const int c = static_cast<int>(i % kChunks);
-    const uint32_t hs = i / kChunks;
-    const int h = static_cast<int>(hs % static_cast<uint32_t>(a.n_heads));
-    const int sl = static_cast<int>(hs / static_cast<uint32_t>(a.n_heads));
+    const int sl = static_cast<int>(i / kChunks);
     const int t = a.idx[static_cast<int64_t>(b) * a.n_slots + sl];
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (t >= 0)
-        v = __ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(a.src) + t * a.src_t +
-                                                   h * a.src_h + c * 8));
-    *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.dst) + b * a.dst_b + sl * a.dst_s + h * a.dst_h + c * 8) = v;
-    if (a.dst_pos && h == 0 && c == 0) {
+    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(a.dst) + b * a.dst_b + sl * a.dst_s + c * 8;
+    if (a.dst_pos && c == 0) {
         float *pd = a.dst_pos + b * a.pos_b + 3 * static_cast<int64_t>(sl);
         for (int e = 0; e < 3; ++e) pd[e] = t >= 0 ? a.src_pos[3 * static_cast<int64_t>(t) + e] : 0.f;
+    }
+    if (t < 0) {
+        for (int h = 0; h < a.n_heads; ++h) *reinterpret_cast<uint4 *>(dst + h * a.dst_h) = make_uint4(0, 0, 0, 0);
+        return;
+    }
+    const __nv_bfloat16 *src = static_cast<const __nv_bfloat16 *>(a.src) + t * a.src_t + c * 8;
+    float cs[4], sn[4];
+    if constexpr (kRope) {
+        const float *pp = a.src_pos + 3 * static_cast<int64_t>(t);
+        token_rotation(s_theta, tab, c, pp[0], pp[1], pp[2], a.out_scale, cs, sn);
+    }
+    for (int h0 = 0; h0 < a.n_heads; h0 += kGatherHeads) {
+        uint4 u[kGatherHeads];
+#pragma unroll
+        for (int j = 0; j < kGatherHeads; ++j)
+            u[j] = h0 + j < a.n_heads ? __ldg(reinterpret_cast<const uint4 *>(src + (h0 + j) * a.src_h))
+                                      : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int j = 0; j < kGatherHeads; ++j) {
+            if (h0 + j >= a.n_heads) break;
+            uint4 v = u[j];
+            if constexpr (kRope) v = rotate8(v, cs, sn);
+            *reinterpret_cast<uint4 *>(dst + (h0 + j) * a.dst_h) = v;
+        }
     }
 }
 
 // dst[idx][h][:] = src[b][s][h][:] for idx >= 0 (dst/src roles of GatherArgs:
-// src is the slotted layout here, dst the token list)
+// src is the slotted layout here, dst the token list); same thread layout.
 template <int D>
 __global__ void __launch_bounds__(256) scatter_kernel(const GatherArgs a) {
     constexpr int kChunks = D / 8;
@@ -358,42 +436,47 @@ __global__ void __launch_bounds__(256) scatter_kernel(const GatherArgs a) {
     if (i >= static_cast<uint32_t>(a.total)) return;
     const int b = blockIdx.y;
     const int c = static_cast<int>(i % kChunks);
-    const uint32_t hs = i / kChunks;
-    const int h = static_cast<int>(hs % static_cast<uint32_t>(a.n_heads));
-    const int sl = static_cast<int>(hs / static_cast<uint32_t>(a.n_heads));
+    const int sl = static_cast<int>(i / kChunks);
     const int t = a.idx[static_cast<int64_t>(b) * a.n_slots + sl];
     if (t < 0) return;
-    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(a.src) + b * a.dst_b +
-                                                          sl * a.dst_s + h * a.dst_h + c * 8));
-    *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.dst) + t * a.src_t + h * a.src_h + c * 8) = v;
+    const __nv_bfloat16 *src = static_cast<const __nv_bfloat16 *>(a.src) + b * a.dst_b + sl * a.dst_s + c * 8;
+    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(a.dst) + t * a.src_t + c * 8;
+    for (int h0 = 0; h0 < a.n_heads; h0 += kGatherHeads) {
+        uint4 u[kGatherHeads];
+#pragma unroll
+        for (int j = 0; j < kGatherHeads; ++j)
+            u[j] = h0 + j < a.n_heads ? __ldg(reinterpret_cast<const uint4 *>(src + (h0 + j) * a.dst_h))
+                                      : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int j = 0; j < kGatherHeads; ++j) {
+            if (h0 + j >= a.n_heads) break;
+            *reinterpret_cast<uint4 *>(dst + (h0 + j) * a.src_h) = u[j];
+        }
+    }
 }
 
 template <int D>
 int gather_launch(const GatherLaunch &l) {
     GatherArgs a{l.dst, l.src, l.idx, l.src_pos, l.dst_pos, l.n_slots, l.n_heads,
                  l.src_t, l.src_h, l.dst_b, l.dst_s, l.dst_h, l.pos_b,
-                 static_cast<int64_t>(l.n_slots) * l.n_heads * (D / 8)};
+                 static_cast<int64_t>(l.n_slots) * (D / 8), l.out_scale};
     if (a.total > 0x7fffffff || l.n_batch > 65535)
         return set_error(SR_ERR_INVALID_ARG, "gather/scatter: too many slots or batch entries");
     const dim3 grid(static_cast<unsigned>((a.total + 255) / 256), l.n_batch);
-    if (l.scatter)
+    if (l.scatter) {
         scatter_kernel<D><<<grid, 256, 0, l.stream>>>(a);
-    else
-        gather_kernel<D><<<grid, 256, 0, l.stream>>>(a);
+    } else if (l.rope) {
+        gather_kernel<D, true><<<grid, 256, 0, l.stream>>>(a, make_rope_table(l.cfg));
+    } else {
+        gather_kernel<D, false><<<grid, 256, 0, l.stream>>>(a, RopeTable{});
+    }
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? SR_OK : set_cuda_error("gather/scatter launch", e);
 }
 
 template <int D, bool kNorm>
 int rope_launch(const RopeLaunch &l) {
-    RopeTable tab{};
-    const int widths[3] = {l.cfg.d_t, l.cfg.d_h, l.cfg.d_w};
-    int pair = 0;
-    for (int ax = 0; ax < 3; ++ax)
-        for (int j = 0; j < widths[ax] / 2; ++j, ++pair)
-            tab.theta[pair] = std::pow(static_cast<double>(l.cfg.base), -2.0 * static_cast<double>(j) / widths[ax]);
-    tab.pairs_t = l.cfg.d_t / 2;
-    tab.pairs_th = (l.cfg.d_t + l.cfg.d_h) / 2;
+    const RopeTable tab = make_rope_table(l.cfg);
     RopeArgs a{static_cast<const __nv_bfloat16 *>(l.x), static_cast<__nv_bfloat16 *>(l.y), l.pos, l.n_valid,
                l.n_heads, l.out_scale, l.xb, l.xt, l.xh, l.yb, l.yt, l.yh, l.pb,
                l.gamma, l.eps, static_cast<__nv_bfloat16 *>(l.y_raw), l.rb, l.rt, l.rh};

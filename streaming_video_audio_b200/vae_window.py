@@ -18,9 +18,10 @@ position differences); a window's tokens are packed valid-first (attention is
 invariant to key order), so partial windows at the grid edge are ragged
 segments.
 
-Everything runs in the library's kernels: sr_gather_tokens (partition),
-sr_rope3d_apply (positions, cache write), sr_chunk_attention_fwd (attention:
-batch = windows, segments = ring slots) and sr_scatter_tokens (merge).
+Everything runs in the library's kernels: sr_gather_tokens (V into the
+ring), sr_gather_rope3d_tokens (K into the ring and the queries into their
+windows, rotated on the way), sr_chunk_attention_fwd (attention: batch =
+windows, segments = ring slots) and sr_scatter_tokens (merge).
 """
 from __future__ import annotations
 
@@ -81,13 +82,9 @@ class RingWindowAttention:
         self.k_ring = torch.zeros(W, H, self.slots * S, D, dtype=torch.bfloat16, **kw)
         self.v_ring = torch.zeros(W, H, self.slots * S, D, dtype=torch.bfloat16, **kw)
         self.q_cap = self.fpc * S
-        self.q_tmp = torch.zeros(W, self.q_cap, H, D, dtype=torch.bfloat16, **kw)
-        self.k_tmp = torch.zeros(W, S, H, D, dtype=torch.bfloat16, **kw)
         self.q_att = torch.zeros(W, H, self.q_cap, D, dtype=torch.bfloat16, **kw)
         self.o_win = torch.zeros(W, self.q_cap, H, D, dtype=torch.bfloat16, **kw)
         self.lse = torch.zeros(W, H, self.q_cap, dtype=torch.float32, **kw)
-        self.pos_q = torch.zeros(W, self.q_cap, 3, dtype=torch.float32, **kw)
-        self.pos_k = torch.zeros(W, S, 3, dtype=torch.float32, **kw)
         self.status = torch.zeros(1, dtype=torch.int32, **kw)
         self.idx_q = torch.from_numpy(self.part.frame_index(self.fpc)).to(self.device)
         per = self.part.gh * self.part.gw
@@ -124,22 +121,20 @@ class RingWindowAttention:
         return (self.calls * self.fpc) % self.slots, min(self.calls, len(self.kv_len_phase) - 1)
 
     def _prepare(self, q, k, v, slot0: int, stream=None) -> None:
-        """Positions, cache write of the current frames' K (RoPE) and V, partition
-        and RoPE of the queries."""
+        """Positions, then the cache write of the current frames (V copied, K
+        rotated on the way into its ring slot) and the partition of the
+        queries (rotated on the way): one gather launch each."""
         S = self.slot_cap
         torch.addcmul(self.pos_base, self.t_axis, self.t0_dev, out=self.pos_cur)
         for f in range(self.fpc):
             sl = (slot0 + f) % self.slots
-            ring_k = self.k_ring[:, :, sl * S:(sl + 1) * S]
-            ring_v = self.v_ring[:, :, sl * S:(sl + 1) * S]
-            # V straight into its ring slot; K through a staging buffer for its one-time RoPE
-            self._gather(ring_v.permute(0, 2, 1, 3), v, self.idx_kv[f], stream=stream)
-            self._gather(self.k_tmp, k, self.idx_kv[f], pos=self.pos_cur, pos_out=self.pos_k, stream=stream)
-            capi.sr_rope3d_apply(self.k_tmp, ring_k.permute(0, 2, 1, 3), self.pos_k, self.split, self.base,
-                                 stream=stream)
-        self._gather(self.q_tmp, q, self.idx_q, pos=self.pos_cur, pos_out=self.pos_q, stream=stream)
-        capi.sr_rope3d_apply(self.q_tmp, self.q_att.permute(0, 2, 1, 3), self.pos_q, self.split, self.base,
-                             stream=stream)
+            ring_k = self.k_ring[:, :, sl * S:(sl + 1) * S].permute(0, 2, 1, 3)
+            ring_v = self.v_ring[:, :, sl * S:(sl + 1) * S].permute(0, 2, 1, 3)
+            capi.sr_gather_tokens(ring_v, v, self.idx_kv[f], stream=stream)
+            capi.sr_gather_rope3d_tokens(ring_k, k, self.idx_kv[f], self.pos_cur, self.split, self.base,
+                                         stream=stream)
+        capi.sr_gather_rope3d_tokens(self.q_att.permute(0, 2, 1, 3), q, self.idx_q, self.pos_cur, self.split,
+                                     self.base, stream=stream)
 
     def _attend(self, phase: int, stream=None) -> None:
         S = self.slot_cap
@@ -203,7 +198,3 @@ class RingWindowAttention:
         gs[2].replay()
         self.calls += 1
         return out
-
-    def _gather(self, dst, src, idx, pos=None, pos_out=None, stream=None):
-        """dst [W, slots, H, D] view <- src tokens [T, H, D] by idx [W, slots]."""
-        capi.sr_gather_tokens(dst, src, idx, src_pos=pos, dst_pos=pos_out, stream=stream)

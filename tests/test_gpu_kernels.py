@@ -291,6 +291,68 @@ def test_qknorm_rope_matches_oracle(D, split, H, N):
         assert_rope_close(y[b].permute(1, 0, 2).cpu(), ref, torch.from_numpy(u))
 
 
+# ---------------------------------------------------------------- gather / scatter (window partition)
+def _gather_case(B, S, T, seed):
+    """idx [B, S]: distinct source tokens with -1 holes (slot order shuffled)."""
+    rng = np.random.default_rng(seed)
+    idx = np.full((B, S), -1, dtype=np.int32)
+    perm = rng.permutation(T)
+    k = 0
+    for b in range(B):
+        n = min(S, T - k, int(rng.integers(S // 2, S + 1)))
+        slots = np.sort(rng.choice(S, size=n, replace=False))
+        idx[b, slots] = perm[k:k + n]
+        k += n
+    return idx
+
+
+@pytest.mark.parametrize("D,H", [(128, 4), (128, 12), (64, 3)])
+def test_gather_and_scatter_tokens_exact(D, H):
+    B, S, T = 5, 40, 170
+    src = workloads.draw_tensor((T, H, D), seed=140)
+    pos = workloads.draw_positions(T, seed=141)
+    idx = _gather_case(B, S, T, seed=142)
+    dst = torch.full((B, S, H, D), 3.0, dtype=torch.bfloat16, device=DEV)
+    dpos = torch.full((B, S, 3), 5.0, device=DEV)
+    capi.sr_gather_tokens(dst, src.to(DEV), torch.from_numpy(idx).to(DEV), src_pos=pos.to(DEV), dst_pos=dpos)
+    back = torch.full((T, H, D), 9.0, dtype=torch.bfloat16, device=DEV)
+    capi.sr_scatter_tokens(back, dst, torch.from_numpy(idx).to(DEV))
+    torch.cuda.synchronize()
+    d, p, bk = dst.cpu(), dpos.cpu(), back.cpu()
+    for b in range(B):
+        for s_ in range(S):
+            t = int(idx[b, s_])
+            if t >= 0:
+                assert torch.equal(d[b, s_], src[t]) and torch.equal(p[b, s_], pos[t])
+            else:
+                assert not d[b, s_].any() and not p[b, s_].any()
+    hit = np.zeros(T, bool)
+    hit[idx[idx >= 0]] = True
+    assert torch.equal(bk[torch.from_numpy(hit)], src[torch.from_numpy(hit)])
+    assert bool((bk[torch.from_numpy(~hit)] == 9.0).all())
+
+
+@pytest.mark.parametrize("D,split,H", [(128, (32, 48, 48), 4), (128, (32, 48, 48), 10), (64, (16, 24, 24), 2)])
+def test_gather_rope3d_tokens_matches_oracle(D, split, H):
+    """The gathered rows rotated by their source token's position: within the
+    RoPE tolerance of the fp64 oracle; holes are zero."""
+    B, S, T = 4, 48, 150
+    src = workloads.draw_tensor((T, H, D), seed=150)
+    pos = workloads.draw_positions(T, seed=151)
+    pos[:, 0] = torch.round(pos[:, 0] * 20) / 20
+    idx = _gather_case(B, S, T, seed=152)
+    dst = torch.full((B, H, S, D), 3.0, dtype=torch.bfloat16, device=DEV)   # head-major, as the ring
+    capi.sr_gather_rope3d_tokens(dst.permute(0, 2, 1, 3), src.to(DEV), torch.from_numpy(idx).to(DEV), pos.to(DEV),
+                                 split)
+    torch.cuda.synchronize()
+    got = dst.permute(0, 2, 1, 3).cpu()
+    sel = idx >= 0
+    rows = idx[sel]
+    ref = oracle.rope3d(src[rows], pos[rows].double(), split)
+    assert_rope_close(got[torch.from_numpy(sel)], ref, src[rows])
+    assert not got[torch.from_numpy(~sel)].any()
+
+
 # ---------------------------------------------------------------- windowed attention (causal VAE decoder)
 @pytest.mark.parametrize("D,split,shift", [(64, (16, 24, 24), 0), (64, (16, 24, 24), 8), (128, (32, 48, 48), 8)])
 def test_ring_window_attention_matches_oracle(D, split, shift):
