@@ -213,10 +213,11 @@ __global__ void __launch_bounds__(128, kPasses <= 5 ? 8 : 4) rope3d_kernel(const
         }
         *reinterpret_cast<uint4 *>(yt + h * a.yh) = pack8(r);
     }
-    if constexpr (kNorm) return;   // the host guarantees n_heads fits the passes above
-    for (int h = hp + kPasses * kHeadsPerPass; h < a.n_heads; h += kHeadsPerPass)   // very many heads
-        *reinterpret_cast<uint4 *>(yt + h * a.yh) =
-            rotate8(__ldg(reinterpret_cast<const uint4 *>(xt + h * a.xh)), cs, sn);
+    if constexpr (!kNorm) {   // with normalisation the host guarantees n_heads fits the passes above
+        for (int h = hp + kPasses * kHeadsPerPass; h < a.n_heads; h += kHeadsPerPass)   // very many heads
+            *reinterpret_cast<uint4 *>(yt + h * a.yh) =
+                rotate8(__ldg(reinterpret_cast<const uint4 *>(xt + h * a.xh)), cs, sn);
+    }
 }
 
 // ============================================================== pooling
