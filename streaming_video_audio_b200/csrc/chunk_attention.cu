@@ -433,26 +433,33 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0 && n_tiles > 0) {
                 constexpr uint32_t idesc_qk = umma_idesc_bf16(kTileM, kTileN, false, false);
                 constexpr uint32_t idesc_pv = umma_idesc_bf16(kTileM, D, false, true);
-                const uint32_t q_base = smem_u32(smem + L::kQ);
-                const uint32_t k_base = smem_u32(smem + L::kK);
-                const uint32_t v_base = smem_u32(smem + L::kV);
+                // Descriptors are built once; each instruction only advances the
+                // start address (one add): the issuing thread shares its SM
+                // sub-partition with busy softmax warps, so its instruction
+                // count matters.
+                const uint64_t desc_q = umma_desc_sw128(smem_u32(smem + L::kQ), 16, 1024);
+                const uint64_t desc_k = umma_desc_sw128(smem_u32(smem + L::kK), 16, 1024);
+                const uint64_t desc_v = umma_desc_sw128(smem_u32(smem + L::kV), kPanelBytes, 1024);
                 auto issue_qk = [&](int t, int st) {
+                    const uint64_t a0 = umma_desc_advance(desc_q, t * L::kTileBytes);
+                    const uint64_t b0 = umma_desc_advance(desc_k, st * L::kTileBytes);
+                    const uint32_t d = tmem + tmem_s(t);
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint32_t off = (kk >> 2) * kPanelBytes + (kk & 3) * 32;
-                        const uint64_t a = umma_desc_sw128(q_base + t * L::kTileBytes + off, 16, 1024);
-                        const uint64_t bd = umma_desc_sw128(k_base + st * L::kTileBytes + off, 16, 1024);
-                        umma_bf16_ss(tmem + tmem_s(t), a, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                        umma_bf16_ss(d, umma_desc_advance(a0, off), umma_desc_advance(b0, off), idesc_qk,
+                                     kk > 0 ? 1u : 0u);
                     }
                     umma_commit(&s_full[t]);
                 };
                 auto issue_pv = [&](int t, int st, bool acc) {
+                    const uint64_t b0 = umma_desc_advance(desc_v, st * L::kTileBytes);
+                    const uint32_t d = tmem + tmem_o(t);
+                    const uint32_t a = tmem + tmem_s(t);
 #pragma unroll
-                    for (int kk = 0; kk < kTileN / 16; ++kk) {
-                        const uint64_t bd = umma_desc_sw128(v_base + st * L::kTileBytes + kk * 2048, kPanelBytes, 1024);
-                        umma_bf16_ts(tmem + tmem_o(t), tmem + tmem_s(t) + kk * 8, bd, idesc_pv,
+                    for (int kk = 0; kk < kTileN / 16; ++kk)
+                        umma_bf16_ts(d, a + kk * 8, umma_desc_advance(b0, kk * 2048), idesc_pv,
                                      (acc || kk > 0) ? 1u : 0u);
-                    }
                     umma_commit(&o_done[t]);
                 };
                 bool ok = mbar_wait(q_full, 0, abort_flag, p.status) && mbar_wait(&k_full[0], 0, abort_flag, p.status);

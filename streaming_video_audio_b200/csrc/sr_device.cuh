@@ -134,6 +134,17 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo
     return d;
 }
 
+// The same descriptor for an operand `bytes` further on in shared memory: only
+// the start-address field (bits 0-13, 16-byte units) changes, and it cannot
+// carry out of its 14 bits because shared-memory addresses stay below 256 KB,
+// so one 32-bit add on the low word does it (the MMA issuer runs this per
+// instruction, instead of rebuilding the whole descriptor).
+__device__ __forceinline__ uint64_t umma_desc_advance(uint64_t d, uint32_t bytes) {
+    const uint32_t lo = static_cast<uint32_t>(d) + (bytes >> 4);
+    const uint32_t hi = static_cast<uint32_t>(d >> 32);
+    return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 accumulation.
 // a_mn / b_mn select MN-major operands.
 __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
