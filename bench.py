@@ -465,6 +465,8 @@ def main():
     ap.add_argument("--config", type=int, default=3, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--impl", default="sr", choices=["sr", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graphs", dest="graphs", action="store_false",
+                    help="launch the step's kernels one by one instead of replaying CUDA graphs")
     ap.add_argument("--row", default="step", choices=["step", "moving", "qknorm", "window", "ulysses"],
                     help="step: the default streaming step; others: the further rows (one JSON line each)")
     args = ap.parse_args()
@@ -506,6 +508,9 @@ def main():
     k_clean, v_clean = k[:, :n_video], v[:, :n_video]   # stand-in for the finished chunk's clean K/V
 
     def one_step(i, ev=None):
+        if args.graphs:   # the step replayed from CUDA graphs (one set per ring state)
+            win.graph_step(q, k, v, k_clean if tiered else None, v_clean if tiered else None, marks=ev)
+            return
         if tiered:
             win.advance(k_clean, v_clean)
         win.append_chunk(k, v)
@@ -516,6 +521,11 @@ def main():
         if ev is not None:
             ev[1].record(stream)
 
+    if args.graphs and tiered:
+        # every ring state is captured during warm-up: the slide cycles through
+        # `period` states, the first call only sets the rings up
+        win.advance(k_clean, v_clean)           # ring set-up (positions of the next state)
+        W = max(W, win.period + 1)
     for i in range(W):
         one_step(i)
     torch.cuda.synchronize()

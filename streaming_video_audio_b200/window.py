@@ -564,6 +564,13 @@ class StreamingWindow:
         elif n != self.slide_frames:
             raise ValueError(f"every slide must move {self.slide_frames} frames")
         ops, nxt = self.slide_ops(self.ring_ptr)
+        self._launch_slide(ops, k_clean, v_clean, stream)
+        self.ring_ptr = nxt
+        self.pos = self._phases[tuple(nxt.values())]
+
+    def _launch_slide(self, ops, k_clean, v_clean, stream=None) -> None:
+        """The kernel calls of one slide plan (no host state changes)."""
+        ft = self.plans[0].frame_tokens
         for op in ops:
             if op[0] == "pool":
                 _, src, fs, dst, fd, m, grid, pool = op
@@ -573,12 +580,52 @@ class StreamingWindow:
                                          self._ring_frames(self.v, dst, fd, m), grid, pool, stream=stream)
             else:
                 _, fr, fc, m = op
-                ft = plan.frame_tokens
                 capi.sr_kv_append(self.k_raw, self.v, None, self.seg["recent"][0] + fr * ft,
                                   k_clean[:, fc * ft:(fc + m) * ft], v_clean[:, fc * ft:(fc + m) * ft], None,
                                   stream=stream)
-        self.ring_ptr = nxt
-        self.pos = self._phases[tuple(nxt.values())]
+
+    def graph_step(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, k_clean: torch.Tensor = None,
+                   v_clean: torch.Tensor = None, marks=None) -> torch.Tensor:
+        """advance(k_clean, v_clean) (when given) and step(q, k, v), replayed
+        from CUDA graphs: no per-launch host work, and the launches follow
+        each other without gaps.
+
+        The tensors must be the same (addresses) on every call.  Each ring
+        state is captured the first time it occurs, after that call has run
+        eagerly; later calls replay two graphs on the current stream (the
+        slide, append and RoPE; the attention), with `marks` recorded around
+        the second.  Returns the window's output buffer."""
+        slide = k_clean is not None
+        key = tuple(self.ring_ptr.values()) if slide and hasattr(self, "rings") else None
+        graphs = self.__dict__.setdefault("_step_graphs", {})
+        if key not in graphs:
+            if slide:
+                self.advance(k_clean, v_clean)
+            self.step(q, k, v, marks=marks)
+            torch.cuda.synchronize()
+            if slide and key is None:    # the rings were set up by this first slide: capture from the next one
+                return self.o
+            ops = self.slide_ops(dict(zip(self.rings, key)))[0] if slide else []
+            g_prep, g_attn = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_prep):   # self.pos already holds the next state's table
+                if slide:
+                    self._launch_slide(ops, k_clean, v_clean)
+                self.append_chunk(k, v)
+                self.rotate(q)
+            with torch.cuda.graph(g_attn):
+                self.attend()
+            graphs[key] = (g_prep, g_attn)
+            return self.o
+        g_prep, g_attn = graphs[key]
+        if slide:
+            nxt = self.slide_ops(self.ring_ptr)[1]
+            self.ring_ptr = nxt
+            self.pos = self._phases[tuple(nxt.values())]
+        g_prep.replay()
+        _mark(marks, 0, None)
+        g_attn.replay()
+        _mark(marks, 1, None)
+        return self.o
 
     def recent_slot_order(self) -> List[int]:
         """Recent frames in chronological order -> their ring slots."""

@@ -279,3 +279,33 @@ def test_window_slide_matches_oracle(n_frames):
                 else:
                     err = np.abs(got.double().numpy() - ref)
                     assert np.all(err <= 2.0 ** -9 * (amax[name] + np.abs(ref)) + 1e-12), (i, role, name)
+
+
+def test_graph_step_matches_eager_steps():
+    """The streaming step replayed from CUDA graphs (slide + append + RoPE,
+    attention) gives the eager sequence advance -> step bit for bit, over
+    more than a full period of ring states (inputs changed in place)."""
+    spec = workloads.scaled(workloads.CHUNK_TIERED, n_heads=2)
+    n = spec.chunk_video_tokens
+    inp = workloads.draw_session(spec, 6)
+    chunks = [tuple(workloads.draw_tensor((1, spec.chunk_len, 2, 128), seed=90 + 3 * s + j) for j in range(3))
+              for s in range(15)]
+    eager = StreamingWindow([spec])
+    eager.load_window([inp])
+    graphed = StreamingWindow([spec])
+    graphed.load_window([inp])
+    q, k, v = (torch.zeros(1, spec.chunk_len, 2, 128, dtype=torch.bfloat16, device="cuda") for _ in range(3))
+    kc = torch.zeros(1, n, 2, 128, dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    for s_, (cq, ck, cv) in enumerate(chunks):
+        clean = chunks[s_ - 1] if s_ else chunks[-1]
+        eager.advance(clean[1][:, :n].cuda(), clean[2][:, :n].cuda())
+        ref = eager.step(cq.cuda(), ck.cuda(), cv.cuda()).cpu()
+        for dst, src in ((q, cq), (k, ck), (v, cv), (kc, clean[1][:, :n]), (vc, clean[2][:, :n])):
+            dst.copy_(src)
+        out = graphed.graph_step(q, k, v, kc, vc).cpu()
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref), s_
+        assert graphed.ring_ptr == eager.ring_ptr
+    graphed.check_status()
+    assert len(graphed._step_graphs) == eager.period
