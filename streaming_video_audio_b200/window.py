@@ -202,6 +202,7 @@ class StreamingWindow:
         if hasattr(self, "rings"):   # a reload restarts the window slide
             self.pos = self._pos_loaded
             del self.rings
+        self.__dict__.pop("_step_graphs", None)   # captured against the old ring state and position tables
         for b, (plan, inp) in enumerate(zip(self.plans, inputs)):
             kb, vb, pb = self.k_raw[b:b + 1], self.v[b:b + 1], self.pos[b:b + 1]
             lp = plan.lengths["prompt"]
