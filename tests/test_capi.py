@@ -8,7 +8,8 @@ import pytest
 from streaming_video_audio_b200 import capi
 
 EXPECTED = {"sr_version", "sr_get_last_error", "sr_rope3d_apply", "sr_history_compress", "sr_kv_append",
-            "sr_chunk_attention_fwd", "sr_chunk_attention_workspace_bytes", "sr_qknorm_rope3d_apply"}
+            "sr_chunk_attention_fwd", "sr_chunk_attention_workspace_bytes", "sr_qknorm_rope3d_apply",
+            "sr_gather_tokens", "sr_gather_rope3d_tokens", "sr_scatter_tokens", "sr_chunk_attention_fwd_noalloc"}
 
 
 def test_header_declares_the_boundary():
@@ -71,6 +72,27 @@ def test_append_and_pool_reject_bad_arguments_on_host():
     rc = lib.sr_history_compress(16, None, 48, 64, 1, 1, 2, 128, cfg, 0, 0, 256, 128, 0, 0, 256, 128,
                                  None, None, 0, None, None)
     assert rc == capi.SR_ERR_INVALID_ARG
+
+
+def test_gather_and_scatter_reject_bad_arguments_on_host():
+    lib = capi.load()
+    cfg = capi.sr_rope_cfg(10000.0, 32, 48, 48)
+    # dst, src, idx, src_pos, B, S, H, D, cfg, scale, src_t, src_h, dst_b, dst_s, dst_h, stream
+    def rope(dst=16, src=32, idx=48, pos=64, S=10, D=128, c=cfg, ts=512):
+        # dst, src, idx, src_pos, B, S, H, D, cfg, scale, src_t, src_h, dst_b, dst_s, dst_h, stream
+        return lib.sr_gather_rope3d_tokens(dst, src, idx, pos, 2, S, 4, D, c, 1.0, ts, 128, 5120, 512, 128, None)
+
+    assert rope(pos=None) == capi.SR_ERR_INVALID_ARG and "src_pos" in _err(lib)
+    assert rope(c=capi.sr_rope_cfg(10000.0, 32, 48, 40)) == capi.SR_ERR_INVALID_ARG
+    assert rope(D=96) == capi.SR_ERR_UNSUPPORTED
+    assert rope(dst=24) == capi.SR_ERR_INVALID_ARG and "aligned" in _err(lib)
+    assert rope(ts=500) == capi.SR_ERR_INVALID_ARG                        # stride not a multiple of 8
+    assert rope(idx=None) == capi.SR_ERR_INVALID_ARG and "null" in _err(lib)
+    assert rope(S=0) == capi.SR_OK                                         # zero work: nothing launched
+    # gather: positions must come as a pair; scatter: null source
+    assert lib.sr_gather_tokens(16, 32, 48, 2, 10, 4, 128, 512, 128, 5120, 512, 128, 64, None, 0, None) == \
+        capi.SR_ERR_INVALID_ARG
+    assert lib.sr_scatter_tokens(16, None, 48, 2, 10, 4, 128, 512, 128, 5120, 512, 128, None) == capi.SR_ERR_INVALID_ARG
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
