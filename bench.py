@@ -1,6 +1,7 @@
 """Benchmark of the chunk-streaming joint video+audio attention step on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config {2,3,4,5}] [--impl {sr,reference}]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config {1..5}] [--impl {sr,reference}]
+                    [--no-graphs] [--no-cpu-baseline] [--row {step,moving,qknorm,window,ulysses}]
 
 A step is one pass of the whole hot path on one batch of synthetic inputs
 resident in HBM: the window slide of the tiered configs (a1: the frames that
@@ -10,16 +11,25 @@ the chunk queries and of every window key (a3) and the fused chunk attention
 (a4).  Default workload: the tiered streaming chunk (config 3), the one
 config on which all four steps run.
 
+The step is replayed from CUDA graphs (one pair per ring state, all
+captured during warm-up); --no-graphs launches its kernels one by one.
+
 Printed: ONE JSON line (rank 0) with attention TFLOP/s of the whole job
 (algorithmic FLOPs 4*Lq*Lkv*D per head over valid tokens only, summed over
 ranks, divided by the max-over-ranks time of K steps), ms per step, the
-attention kernel's roofline (CUDA events on the launch stream), clocks
-sampled during the timed region, an end-to-end figure through
-``StreamingWindow.step_from_host`` (pinned host buffers, copies inside the
-timed region) and the fp64 oracle timed on a bounded sample on the host.
+attention kernel's roofline (CUDA events on the launch stream; the burst
+bf16 peak for a short timed region, the sustained one from 0.5 s on), clocks
+sampled inside the timed region, an end-to-end figure through
+``HostStepPipeline`` (pinned host buffers, host<->device copies inside the
+timed region, overlapped with compute) and the fp64 oracle timed on a
+bounded sample on the host.  --row measures one of the further rows instead
+(prefix / moving part, fused QK-norm + RoPE, the causal VAE decoder's ring
+window attention, Ulysses), one JSON line each.
 
 Multi-GPU (torchrun): every rank runs its own sessions (seed offset by
-rank); there is no data-path collective (weak scaling).
+rank); there is no data-path collective (weak scaling).  --row ulysses
+splits one session over the ranks instead (strong scaling, two NCCL
+all-to-alls per step).
 """
 from __future__ import annotations
 
