@@ -1,5 +1,8 @@
 """Streaming window: persistent per-layer KV buffers, their segment layout and
-the window position template, plus the four-call streaming step.
+the window position template; the streaming step (KV append, RoPE,
+attention), the window slide after a chunk (tier re-pooling over frame
+rings), the prefix / moving-part split, CUDA-graph replay of the step and a
+host-buffer pipeline.
 
 Sources:
   * "StreamRender-H3" (molayo1419.me), streaming context section: a sink
@@ -20,7 +23,11 @@ chunk's frames at t = 0, 1, ... and the context frames at t = -n .. -1 (the
 sink earliest); audio token i at t = i * 6 / 40, h = w = 0; pooled cells at
 (t, mean member row, mean member col); the prompt unrotated; K is kept
 pre-RoPE in the window (``k_raw``) and rotated into ``k_att`` with the current
-template, so re-positioning never compounds rounding.
+template, so re-positioning never compounds rounding.  After a chunk its
+clean frames become the newest history and every tier hands its oldest
+frames to the next older tier (re-pooled), the oldest tier dropping its
+oldest: each of tier0.., recent is a ring of frame slots, so only the frames
+that change tier move.
 
 Buffer layout (per session, head-major, the attention kernel's layout):
     [prompt | sink | tier (oldest first) ... | recent | chunk]
