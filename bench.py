@@ -121,8 +121,16 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.p.kill()
         self.f.flush()
-        rows = [r.split(",") for r in open(self.f.name).read().strip().splitlines() if r.strip()]
+        text = open(self.f.name).read()
         os.unlink(self.f.name)
+        return self.summarize(text, *self.window)
+
+    @staticmethod
+    def summarize(text: str, t0=None, t1=None):
+        """Median SM clock, max clock and active throttle reasons of the
+        nvidia-smi CSV lines in `text` (FIELDS order), keeping those stamped
+        within [t0, t1] (host epoch seconds) when there are any."""
+        rows = [r.split(",") for r in text.strip().splitlines() if r.strip()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         samples = []
         for r in rows:
@@ -135,7 +143,6 @@ class ClockSampler:
                 continue
         if not samples:
             return None
-        t0, t1 = self.window
         inside = [x for x in samples if t0 is not None and t1 is not None and t0 <= x[0] <= t1]
         use = inside or samples
         reasons = set().union(*[x[3] for x in use])

@@ -1,0 +1,34 @@
+"""Host-side pieces of bench.py (CPU only): clock-sample summaries and the
+launch count of the timed steps."""
+import time
+
+import bench
+
+
+def _line(ts, sm, reasons=("Not Active",) * 4):
+    stamp = time.strftime("%Y/%m/%d %H:%M:%S", time.localtime(ts)) + ".250"
+    return ", ".join([stamp, "0", str(sm), "1965", "900.00", "0x0"] + list(reasons))
+
+
+def test_clock_summary_keeps_the_timed_window():
+    t = time.time()
+    text = "\n".join([_line(t - 3, 600), _line(t - 1, 1800, ("Not Active", "Not Active", "Not Active", "Active")),
+                      _line(t, 1700), _line(t + 5, 1965)])
+    s = bench.ClockSampler.summarize(text, t - 1.5, t + 1)
+    assert s["samples"] == 2 and s["in_timed_region"]
+    assert s["sm_mhz"] == 1750.0 and s["sm_max_mhz"] == 1965.0 and s["reasons"] == ["sw_power_cap"]
+    s = bench.ClockSampler.summarize(text, t + 10, t + 11)      # window without samples: all, flagged
+    assert s["samples"] == 4 and not s["in_timed_region"]
+    assert bench.ClockSampler.summarize("") is None
+    assert bench.ClockSampler.summarize("garbage line\n") is None
+
+
+def test_launch_count_follows_the_slide_plan():
+    import workloads
+    from streaming_video_audio_b200.window import StreamingWindow
+    spec = workloads.scaled(workloads.CHUNK_TIERED, n_heads=1, head_dim=128, prompt_len=8, chunk_audio_tokens=4)
+    win = StreamingWindow([spec], device="cpu")
+    win._ring_setup(3)
+    # CPU window: no split workspace -> 4 launches per step (append, 2 RoPE, attention) + 3 for the slide
+    assert bench.launches_in_steps(win, True, 10) == 10 * (4 + 3)
+    assert bench.launches_in_steps(win, False, 10) == 40
