@@ -109,3 +109,19 @@ def test_slide_rejects_inputs_it_cannot_place():
     spec = workloads.scaled(workloads.CHUNK, context_video_tokens=4 * FT - 10)
     with pytest.raises(ValueError):
         StreamingWindow([spec], device="cpu")._ring_setup(1)     # partial history frame
+
+
+@pytest.mark.parametrize("config", [1, 2, 3, 4, 5])
+def test_window_layout_and_chunk_positions_match_oracle_on_host(config):
+    """Segment capacities, offsets and the chunk's position template of the
+    product's window (host side) against the oracle's own layout code."""
+    from oracle import layout as olayout
+    specs = [s for s, _ in workloads.session_list(config)]
+    win = StreamingWindow(specs, device="cpu")
+    assert win.caps == olayout.capacities(specs)
+    assert win.offsets == olayout.segment_offsets(olayout.capacities(specs))
+    for b, spec in enumerate(specs):
+        ref = np.asarray(olayout.chunk_positions(spec), dtype=np.float32)
+        assert np.array_equal(win.q_pos[b, :spec.chunk_len].numpy(), ref)
+        assert not win.q_pos[b, spec.chunk_len:].any()
+        assert [int(x) for x in win.lengths[b]] == olayout.segment_lengths(spec)
