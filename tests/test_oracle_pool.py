@@ -157,3 +157,40 @@ def test_window_membership_partitions_the_grid():
         assert sum(len(x) for x in seen.values()) == 20 * 36
         assert all(len(x) <= 256 for x in seen.values())
         assert len(seen) == (-(-(20 + shift) // 16)) * (-(-(36 + shift) // 16))
+
+
+def test_window_reference_sees_only_its_window_and_its_history():
+    """Pins of the ring-window reference: (1) frames older than the history
+    leave the current output unchanged, one frame inside it does not;
+    (2) a token changed in one window leaves every other window's output
+    unchanged and changes its own; (3) the shift moves the window borders."""
+    from oracle import vae_window
+    F, gh, gw, H, D = 5, 20, 20, 1, 64
+    kw = dict(grid_hw=(gh, gw), t0=3, call_frames=2, history=2, split=(16, 24, 24))
+    q = workloads.draw_tensor((F, gh * gw, H, D), seed=21)
+    k = workloads.draw_tensor((F, gh * gw, H, D), seed=22)
+    v = workloads.draw_tensor((F, gh * gw, H, D), seed=23)
+    base = vae_window.window_attention_reference(q, k, v, **kw)
+    # (1) frame 0 is outside the 2-frame history of the call on frames 3, 4; frame 1 is inside
+    k2, v2 = k.clone(), v.clone()
+    k2[0] += 1.0
+    v2[0] -= 2.0
+    assert np.array_equal(vae_window.window_attention_reference(q, k2, v2, **kw), base)
+    v3 = v.clone()
+    v3[1] += 1.0
+    assert not np.allclose(vae_window.window_attention_reference(q, k, v3, **kw), base)
+    # (2) change the value of token (row 2, col 3) of frame 2: window (0, 0) only (no shift)
+    v4 = v.clone()
+    v4[2, 2 * gw + 3] += 5.0
+    out = vae_window.window_attention_reference(q, k, v4, **kw)
+    rows = np.arange(2 * gh * gw) % (gh * gw)
+    in_w00 = ((rows // gw) < 16) & ((rows % gw) < 16)
+    assert np.array_equal(out[~in_w00], base[~in_w00])
+    assert not np.allclose(out[in_w00], base[in_w00])
+    # (3) with shift 8 the same token's window is the corner one: rows and cols [0, 8)
+    kw8 = dict(kw, shift=8)
+    base8 = vae_window.window_attention_reference(q, k, v, **kw8)
+    out8 = vae_window.window_attention_reference(q, k, v4, **kw8)
+    in_w = ((rows // gw) < 8) & ((rows % gw) < 8)
+    assert np.array_equal(out8[~in_w], base8[~in_w])
+    assert not np.allclose(out8[in_w], base8[in_w])
