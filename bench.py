@@ -52,6 +52,8 @@ import torch  # noqa: E402
 
 import workloads  # noqa: E402
 
+METRIC = "chunk attention TFLOP/s and ms per streaming step on 1 B200; fraction of BF16 peak"
+
 CONFIG_DESC = {
     1: "tiny: 1 head x 64, chunk 2x6x8 video + 4 audio over 16 prompt + 2 context frames",
     2: "chunk: one streaming chunk at 1344x768 (3 latent frames x 1008 + 20 audio) over 256 prompt + "
@@ -190,70 +192,204 @@ def build_window(config: int, rank: int, device):
     return specs, inputs, win, chunk
 
 
+# sources of the attention launch at head_dim 128 (pair kernel, dispatch and
+# split merge, device helpers): a traffic record is only used while they are
+# unchanged since its capture
+ATTENTION_SOURCES = ("pair_attention.cu", "chunk_attention.cu", "sr_device.cuh")
+
+
+def attention_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for name in ATTENTION_SOURCES:
+        h.update(open(os.path.join(ROOT, "streaming_video_audio_b200", "csrc", name), "rb").read())
+    return h.hexdigest()[:16]
+
+
 def attention_traffic(config: int):
     """DRAM bytes per attention launch from the committed ncu capture
     (profiles/attention_traffic.json), or None when the capture was taken on
     another workload or the kernel source has changed since."""
-    import hashlib
     path = os.path.join(ROOT, "profiles", "attention_traffic.json")
     if config != 3 or not os.path.exists(path):
         return None
     rec = json.load(open(path))
-    src = os.path.join(ROOT, "streaming_video_audio_b200", "csrc")
-    h = hashlib.sha256()
-    for name in ("chunk_attention.cu", "sr_device.cuh"):
-        h.update(open(os.path.join(src, name), "rb").read())
-    if h.hexdigest()[:16] != rec.get("source_sha256_16"):
+    if attention_source_hash() != rec.get("source_sha256_16"):
         return None
     return int(rec["dram_bytes_read"]) + int(rec["dram_bytes_write"])
 
 
+def call_breakdown(step_marks):
+    """Mean device time and algorithmic bytes per step of every named call,
+    from the (name, bytes, start, end) event lists of graph_step(op_marks=...):
+    calls of one name within a step (a ring wrap splits one into two) are
+    summed, then averaged over the steps."""
+    agg = {}
+    for m in step_marks:
+        per = {}
+        for name, nbytes, a, b in m:
+            d = per.setdefault(name, [0.0, 0])
+            d[0] += a.elapsed_time(b)
+            d[1] += nbytes or 0
+        for name, (ms, nb) in per.items():
+            e = agg.setdefault(name, [0.0, 0, 0])
+            e[0] += ms
+            e[1] += nb
+            e[2] += 1
+    return [(name, ms / cnt, nb / cnt) for name, (ms, nb, cnt) in agg.items()]
+
+
+def hbm_block(breakdown, hbm_peak: float, peak_kind: str, prep_ms: float = None):
+    """roofline.hbm of the bench line: every HBM-bound call of the step with
+    its mean ms, algorithmic bytes, GB/s and fraction of the measured copy
+    bandwidth (and of the 8 TB/s nominal figure), each call timed alone; and,
+    with prep_ms (the part of the timed steps before the attention launch,
+    where independent calls overlap), the same for the calls as one group."""
+    rows = []
+    for name, ms, nb in breakdown:
+        if name == "attention" or ms <= 0 or not nb:   # the clock advance moves no bulk data
+            continue
+        gbs = nb / (ms * 1e-3) / 1e9
+        rows.append({"call": name, "ms": ms, "bytes": int(nb), "achieved": gbs, "frac": gbs / hbm_peak,
+                     "frac_of_8tbs": gbs / 8000.0})
+    tot_b = sum(r["bytes"] for r in rows)
+    tot_ms = sum(r["ms"] for r in rows)
+    return {"bound": "hbm", "unit": "GB/s", "peak": hbm_peak, "peak_kind": f"{peak_kind} copy bandwidth",
+            "calls": rows, "all_calls": {"ms": tot_ms, "bytes": tot_b,
+                                         "achieved": tot_b / (tot_ms * 1e-3) / 1e9 if tot_ms > 0 else None,
+                                         "frac": tot_b / (tot_ms * 1e-3) / 1e9 / hbm_peak if tot_ms > 0 else None},
+            "step_ms_sum_of_calls": sum(ms for _, ms, _ in breakdown),
+            "prep_group": None if prep_ms is None or prep_ms <= 0 else
+            {"ms": prep_ms, "bytes": tot_b, "achieved": tot_b / (prep_ms * 1e-3) / 1e9,
+             "frac": tot_b / (prep_ms * 1e-3) / 1e9 / hbm_peak,
+             "how": "timed steps: step start to the attention launch (independent calls on parallel graph branches)"},
+            "how": "each call replayed from its own CUDA graph, events between calls, after the timed region"}
+
+
 def launches_in_steps(win, tiered: bool, steps: int) -> int:
     """Library kernel launches of `steps` steps from the window's current
-    slide state: append, RoPE of q, RoPE of the window, attention (+ the
-    split merge) per step, and the slide's pooling and append calls."""
+    slide state: append (+ RoPE) of the chunk, RoPE of q, RoPE of the prefix
+    (or of the window), attention (+ the split merge) per step, and the
+    slide's clock advance, pooling and append calls."""
     n = (4 + (1 if win.workspace is not None else 0)) * steps
     if tiered:
         ptr = dict(win.ring_ptr)
         for _ in range(steps):
             ops, ptr = win.slide_ops(ptr)
-            n += len(ops)
+            n += 1 + len(ops)
     return n
 
 
-def cpu_baseline(specs, inputs, target_s: float = 12.0):
-    """The fp64 oracle as it stands, on the host cores: every head of a
-    sample of chunk rows of the first session (window assembly, pooling and
-    RoPE of every key included in each call).  A 64-row probe sizes the
-    measured sample to about target_s seconds of CPU work."""
+def oracle_sample(spec, inp, target_s: float, heads=None):
+    """The fp64 oracle as it stands, on the host cores: the given heads (all by
+    default) of a seeded sample of chunk rows of one session, window assembly,
+    pooling and RoPE of every key included in each call.  Two probes separate
+    the per-call cost from the per-row cost and size one run of about
+    target_s seconds.  Returns (TFLOP/s, rows, seconds, O [rows, heads, D])."""
     import oracle
     from streaming_video_audio_b200.window import SessionPlan
-    spec, inp = specs[0], inputs[0]
     rng = np.random.default_rng(0)
     order = rng.permutation(spec.chunk_len)
 
     def timed(n):
         rows = sorted(order[:n].tolist())
         t0 = time.perf_counter()
-        oracle.session_reference(spec, inp, rows=rows)
-        return rows, time.perf_counter() - t0
+        o, _ = oracle.session_reference(spec, inp, heads=heads, rows=rows)
+        return rows, time.perf_counter() - t0, o
 
-    # two probes separate the per-call cost (window assembly, pooling, RoPE of
-    # every key) from the per-row cost, then one run of about target_s seconds
-    _, t1 = timed(min(64, spec.chunk_len))
-    rows, t2 = timed(min(128, spec.chunk_len))
-    per_row = max((t2 - t1) / 64.0, 1e-4)
-    fixed = max(t1 - 64 * per_row, 0.0)
-    n = int(min(spec.chunk_len, max(128, (target_s - fixed) / per_row)))
+    p1 = min(16, spec.chunk_len)
+    p2 = min(128, spec.chunk_len)
+    _, t1, _ = timed(p1)
+    rows, t2, o = timed(p2)
+    # per-row cost from the difference; a difference lost in noise falls back
+    # to the larger probe's mean (an overestimate: the sample stays bounded)
+    per_row = (t2 - t1) / max(p2 - p1, 1)
+    if per_row <= 0.1 * t2 / p2:
+        per_row = t2 / p2
+    fixed = max(t1 - p1 * per_row, 0.0)
+    n = int(min(spec.chunk_len, max(p2, (target_s - fixed) / per_row)))
     if n > len(rows):
-        rows, dt = timed(n)
+        rows, dt, o = timed(n)
     else:
         dt = t2
     lkv = sum(SessionPlan(spec).lengths.values())
-    fl = 4.0 * len(rows) * lkv * spec.head_dim * spec.n_heads
-    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{len(rows)} of {spec.chunk_len} chunk rows x all {spec.n_heads} heads of {spec.name} "
-                      f"(window assembly, pooling and RoPE of every key included), {dt:.1f} s"}
+    n_heads = spec.n_heads if heads is None else len(heads)
+    fl = 4.0 * len(rows) * lkv * spec.head_dim * n_heads
+    return fl / dt / 1e12, rows, dt, o
+
+
+def run_configs(main_config: int, device, peak: float, n_attn: int = 20, target_s: float = 6.0,
+                others_s: float = 2.0):
+    """Every workload config once, after the timed region: a fresh window on
+    the GPU, one step, the attention launch timed on its own (n_attn launches
+    between CUDA events after 3 warm-up launches), the fp64 oracle timed on a
+    bounded sample of the first session on the host cores (the bench's own
+    config with every head; the 5 s clip and the ragged batch on two heads)
+    and the GPU output compared with that same oracle output (max-abs and
+    mean-abs error per config).  Also the streaming chunk's oracle on one
+    thread.  Returns (per-config dict, cpu_baseline dict)."""
+    import oracle
+    from streaming_video_audio_b200.window import StreamingWindow
+    cores = oracle.num_threads()
+    out = {}
+    for c in (1, 2, 3, 4, 5):
+        sessions = workloads.session_list(c)
+        specs = [sp for sp, _ in sessions]
+        inputs = [workloads.draw_session(sp, seed) for sp, seed in sessions]
+        win = StreamingWindow(specs, device=device)
+        win.load_window(inputs)
+        B, qc, H, D = win.B, win.q_cap, win.H, win.D
+        chunk = []
+        for name in ("q", "k", "v"):
+            t = torch.zeros(B, qc, H, D, dtype=torch.bfloat16)
+            for b, inp in enumerate(inputs):
+                x = getattr(inp, name)
+                t[b, :x.shape[0]] = x
+            chunk.append(t.to(device))
+        win.step(*chunk)
+        torch.cuda.synchronize()
+        win.check_status()
+        o_gpu = win.o[0].double().cpu()
+        for _ in range(3):
+            win.attend()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ev[0].record()
+        for _ in range(n_attn):
+            win.attend()
+        ev[1].record()
+        torch.cuda.synchronize()
+        win.check_status()
+        attn_ms = ev[0].elapsed_time(ev[1]) / n_attn
+        flops = attention_flops(specs)
+        spec, inp = specs[0], inputs[0]
+        heads = None if c in (1, 2, 3) else [0, spec.n_heads // 2]
+        val, rows, dt, ref = oracle_sample(spec, inp, target_s if c == main_config else others_s, heads=heads)
+        sel = list(range(spec.n_heads)) if heads is None else heads
+        err = np.abs(o_gpu[rows][:, sel].numpy() - ref)
+        out[str(c)] = {
+            "workload": spec.name + (f" x{len(specs)} sessions" if len(specs) > 1 else ""),
+            "attention_ms": attn_ms, "attention_tflops": flops / (attn_ms * 1e-3) / 1e12,
+            "frac_of_burst": flops / (attn_ms * 1e-3) / 1e12 / peak,
+            "parity": {"max_abs": float(err.max()), "mean_abs": float(err.mean()), "rows": len(rows),
+                       "heads": len(sel), "session": 0, "bar": [2e-2, 2e-3]},
+            "oracle": {"value": val, "unit": "TFLOP/s", "rows": len(rows), "heads": len(sel), "seconds": dt}}
+        del win, chunk, o_gpu
+        torch.cuda.empty_cache()
+    main = out[str(main_config)]
+    base = {"value": main["oracle"]["value"], "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{main['oracle']['rows']} chunk rows x all {main['oracle']['heads']} heads of the first "
+                      f"session of config {main_config} (window assembly, pooling and RoPE of every key included), "
+                      f"{main['oracle']['seconds']:.1f} s",
+            "per_config": {c: d["oracle"] for c, d in out.items()}}
+    spec, seed = workloads.session_list(2)[0]
+    inp = workloads.draw_session(spec, seed)
+    oracle.set_num_threads(1)
+    try:
+        v, rows, dt, _ = oracle_sample(spec, inp, others_s, heads=[0])
+    finally:
+        oracle.set_num_threads(cores)
+    base["one_thread_config2"] = {"value": v, "rows": len(rows), "heads": 1, "seconds": dt, "cores": 1}
+    return out, base
 
 
 def run_reference(args, rank, world):
@@ -282,7 +418,7 @@ def run_reference(args, rank, world):
     val = fl / dt / 1e12
     cores = oracle.num_threads()
     sample = f"per step: {len(rows)} chunk rows x 1 head of {spec.name} (full window assembly, pooling, RoPE)"
-    line = {"metric": "chunk attention TFLOP/s (fp64 CPU oracle)", "value": val, "unit": "TFLOP/s",
+    line = {"metric": METRIC, "value": val, "unit": "TFLOP/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
@@ -305,12 +441,13 @@ ROW_DESC = {
 }
 
 
-def _timed(step, K, W, local, dist=None, before=None):
-    """W warm-up steps, then K steps between barriers and synchronisations;
-    step(i, marks) records `marks` around its dominant launch; `before` runs
-    on the host between the two.  Returns (total ms, mean dominant-launch ms,
-    clocks)."""
+def _timed(step, K, W, local, dist=None, before=None, capture=0):
+    """`capture` graph-capture steps and W warm-up steps, then K steps between
+    barriers and synchronisations; step(i, marks) records `marks` around its
+    dominant launch; `before` runs on the host between the two.  Returns
+    (total ms, mean dominant-launch ms, clocks)."""
     stream = torch.cuda.current_stream()
+    W = capture + W
     for i in range(W):
         step(i, None)
     torch.cuda.synchronize()
@@ -423,7 +560,6 @@ def run_row(args, rank, world, local, device, dist):
                         .to(device) for j in range(3)) for c in range(2)]
         out = torch.empty(2 * T, H, D, dtype=torch.bfloat16, device=device)
         q_in, k_in, v_in = (torch.empty_like(out) for _ in range(3))
-        W = max(W, 6)    # the 6-frame ring is full after 3 calls; its 6 states are captured as CUDA graphs by then
 
         def step(i, marks):
             # each call's frames arrive in the layer's input buffers (a device copy), then
@@ -432,7 +568,9 @@ def run_row(args, rank, world, local, device, dist):
                 dst.copy_(src)
             layer.graphed(q_in, k_in, v_in, t0=2 * i, out=out, marks=marks)
 
-        total, kern, clocks = _timed(step, K, W, local, dist)
+        # the 6-frame ring is full after 3 calls; its 6 states are captured as
+        # CUDA graphs in a capture phase of 6 calls before the warm-up
+        total, kern, clocks = _timed(step, K, W, local, dist, capture=6)
         assert int(layer.status.item()) == 0
         counts = layer.part.counts.astype(np.float64)
         fl = float(np.sum(4.0 * (2 * counts) * (6 * counts) * D * H))
@@ -441,9 +579,9 @@ def run_row(args, rank, world, local, device, dist):
                 "unit": "TFLOP/s", "frac": ach / peak, "peak_kind": peak_kind, "attention_ms": kern,
                 "traffic": None}
         value = world * fl * K / (total * 1e-3) / 1e12
-        # per frame: gather of V, gather + RoPE of K; gather + RoPE of Q; attention (+ merge);
-        # scatter (plus torch's position add and the three input copies, not counted)
-        launches = K * (2 * 2 + 1 + 1 + 1 + (1 if layer.workspace is not None else 0))
+        # per frame: gather of V, gather + RoPE of K; the frame clock; gather + RoPE of Q;
+        # attention (+ merge); scatter (the three input copies are device-to-device memcpys)
+        launches = K * (2 * 2 + 1 + 1 + 1 + 1 + (1 if layer.workspace is not None else 0))
         return _row_line(args, world, "windowed attention TFLOP/s per decoder call (2 latent frames)", value,
                          "TFLOP/s", total, {"windows": layer.part.n_windows, "tokens_per_call": 2 * T}, roof,
                          clocks, launches)
@@ -473,7 +611,9 @@ def run_row(args, rank, world, local, device, dist):
         roof = {"bound": "tensor", "kernel": "chunk_attention_kernel<128>", "achieved": ach, "peak": peak,
                 "unit": "TFLOP/s", "frac": ach / peak, "peak_kind": peak_kind, "attention_ms": agg["attn_ms"],
                 "traffic": None}
-        launches = K * (4 + (1 if ua.win.workspace is not None else 0))
+        # pack (3 gathers), the window step (append + RoPE, RoPE of q, RoPE of the
+        # prefix, attention (+ merge)), unpack (1 scatter); the all-to-alls are NCCL's
+        launches = K * (3 + 4 + 1 + (1 if ua.win.workspace is not None else 0))
         line = _row_line(args, world, "attention TFLOP/s of one session's streaming step (whole job)",
                          agg["value"], "TFLOP/s", agg["total_ms"],
                          {"heads_per_rank": ua.Hn, "tokens_per_rank": ua.S, "parallelism": f"ulysses{world}",
@@ -550,36 +690,64 @@ def main():
         if ev is not None:
             ev[1].record(stream)
 
-    if args.graphs and tiered:
-        # every ring state is captured during warm-up: the slide cycles through
-        # `period` states, the first call only sets the rings up
-        win.advance(k_clean, v_clean)           # ring set-up (positions of the next state)
-        W = max(W, win.period + 1)
-    for i in range(W):
+    # graph capture is its own phase, before the warm-up: every ring state the
+    # slide cycles through is captured once (the first call only sets the
+    # rings up); the W warm-up steps that follow replay the graphs like the
+    # timed steps do
+    capture_steps = 0
+    if args.graphs:
+        if tiered:
+            win.advance(k_clean, v_clean)           # ring set-up (positions of the next state)
+            capture_steps = win.period
+        else:
+            capture_steps = 1
+    for i in range(capture_steps):
         one_step(i)
+    for i in range(W):
+        one_step(capture_steps + i)
     torch.cuda.synchronize()
     win.check_status()
 
     launches = launches_in_steps(win, tiered, K)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    bounds = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]   # step boundaries
     sampler = ClockSampler(local)
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     sampler.mark(0)
-    start.record(stream)
+    bounds[0].record(stream)
     for i in range(K):
-        one_step(W + i, evs[i])
-    stop.record(stream)
+        one_step(capture_steps + W + i, evs[i])
+        bounds[i + 1].record(stream)
     torch.cuda.synchronize()
     sampler.mark(1)
     if dist:
         dist.barrier()
     clocks = sampler.stop()
     win.check_status()
-    total_ms = start.elapsed_time(stop)
+    total_ms = bounds[0].elapsed_time(bounds[K])
     attn_ms = [a.elapsed_time(b) for a, b in evs]
+    step_ms = np.array([bounds[i].elapsed_time(bounds[i + 1]) for i in range(K)])
+    # everything before the attention launch in each step (the slide, the
+    # appends and the RoPE calls, overlapped where independent)
+    prep_ms = float(np.mean([bounds[i].elapsed_time(evs[i][0]) for i in range(K)]))
+
+    # per-call breakdown of the same step: every library call replayed from a
+    # graph of its own with CUDA events between them (the host enqueues far
+    # ahead of the device, so the events see no launch gaps); HBM roofline of
+    # each call from its algorithmic bytes
+    breakdown = None
+    if args.graphs:
+        n_bd = min(K, 200)
+        marks = []
+        for i in range(n_bd):
+            m = []
+            win.graph_step(q, k, v, k_clean if tiered else None, v_clean if tiered else None, op_marks=m)
+            marks.append(m)
+        torch.cuda.synchronize()
+        win.check_status()
+        breakdown = call_breakdown(marks)
 
     # end to end through the public host-buffer API: every step uploads its
     # q, k, v from pinned host memory and downloads its o; HostStepPipeline
@@ -615,11 +783,14 @@ def main():
     if rank == 0:
         achieved = flops / (attn_avg_ms * 1e-3) / 1e12
         line = {
-            "metric": "chunk attention TFLOP/s and ms per streaming step on 1 B200; fraction of BF16 peak",
+            "metric": METRIC,
             "value": agg["value"],
             "unit": "TFLOP/s",
-            "n_gpus": world, "steps": K, "warmup": W,
+            "n_gpus": world, "steps": K, "warmup": W, "graph_capture_steps": capture_steps,
             "ms_per_step": total_ms / K,
+            # this rank's per-step times (events at every step boundary)
+            "step_ms": {"median": float(np.median(step_ms)), "p10": float(np.percentile(step_ms, 10)),
+                        "p90": float(np.percentile(step_ms, 90)), "mean": float(step_ms.mean())},
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
             "config": {"workload": CONFIG_DESC[args.config], "config": args.config,
@@ -639,7 +810,8 @@ def main():
                          "peak_kind": f"{peak_kind} {'sustained' if total_ms >= 500.0 else 'burst'}",
                          "timed_region_ms": total_ms,
                          "attention_ms": attn_avg_ms, "traffic": attention_traffic(args.config),
-                         "algorithmic_bytes": attention_bytes(win)},
+                         "algorithmic_bytes": attention_bytes(win),
+                         "hbm": hbm_block(breakdown, hbm, peak_kind, prep_ms) if breakdown else None},
             "e2e": {"value": agg["e2e_value"], "unit": "TFLOP/s",
                     "ms_per_step": e2e_ms / K,
                     "h2d_bytes_per_step": sum(t.numel() * 2 for t in chunk),
@@ -648,7 +820,10 @@ def main():
             "gpu_launches": launches,
         }
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(specs, inputs)
+            per_config, base = run_configs(args.config, device, peak)
+            line["cpu_baseline"] = base
+            line["configs"] = per_config
+            line["parity"] = {c: [d["parity"]["max_abs"], d["parity"]["mean_abs"]] for c, d in per_config.items()}
         print(json.dumps(line), flush=True)
     if dist:
         dist.barrier()

@@ -72,6 +72,10 @@ const char *sr_get_last_error(void);
  * y   element (b, n, h, d) at y + b*y_batch_stride + n*y_token_stride + h*y_head_stride + d
  * pos fp32 (t, h, w) of token (b, n) at pos + b*pos_batch_stride + 3*n; NULL = all zero
  *     (a pure re-layout, optionally scaled).
+ * t_origin_dev  optional fp64 on the device added to every token's t before
+ *     the angle is formed (in fp64): the stream clock of a streaming session,
+ *     so that keys rotated at different steps share one time axis.  NULL = 0.
+ *     8-byte aligned.
  * n_valid_dev  optional int32[n_batch] on the device: tokens n >= n_valid[b]
  *     are skipped (neither read nor written).  NULL = all n_tokens.
  * Layouts: any strides, e.g. token-major [B, N, H, D] in, head-major
@@ -89,7 +93,7 @@ int sr_rope3d_apply(const void *x, void *y, const float *pos,
                     const int32_t *n_valid_dev, sr_rope_cfg cfg, float out_scale,
                     int64_t x_batch_stride, int64_t x_token_stride, int64_t x_head_stride,
                     int64_t y_batch_stride, int64_t y_token_stride, int64_t y_head_stride,
-                    int64_t pos_batch_stride, void *stream);
+                    int64_t pos_batch_stride, const double *t_origin_dev, void *stream);
 
 /* QK normalisation fused with the 3-D RoPE and the cache write.
  *
@@ -104,7 +108,8 @@ int sr_rope3d_apply(const void *x, void *y, const float *pos,
  *   y = out_scale * R(pos) u                         (bf16 RNE)
  *   y_raw = u                                        (bf16 RNE, optional)
  * Arguments as in sr_rope3d_apply, plus gamma: fp32 [head_dim] on the device
- * (16-byte aligned); eps >= 0; y_raw: optional output with its own strides
+ * (16-byte aligned); eps >= 0; t_origin_dev as for sr_rope3d_apply; y_raw:
+ * optional output with its own strides
  * (element (b, n, h, d) at y_raw + b*yraw_batch_stride + n*yraw_token_stride
  * + h*yraw_head_stride + d), NULL = not written.
  * Requires n_heads <= 64 at head_dim 128 (<= 128 at head_dim 64).
@@ -115,7 +120,32 @@ int sr_qknorm_rope3d_apply(const void *x, void *y, void *y_raw, const float *gam
                            int64_t x_batch_stride, int64_t x_token_stride, int64_t x_head_stride,
                            int64_t y_batch_stride, int64_t y_token_stride, int64_t y_head_stride,
                            int64_t yraw_batch_stride, int64_t yraw_token_stride, int64_t yraw_head_stride,
-                           int64_t pos_batch_stride, void *stream);
+                           int64_t pos_batch_stride, const double *t_origin_dev, void *stream);
+
+/* Fused rotation of the K that a call writes into the window (optional
+ * argument of sr_kv_append and sr_history_compress): the key enters its slot
+ * rotated once, as sr_rope3d_apply would rotate it,
+ *     k_rot[...] = out_scale * R(pos + (*t_origin_dev, 0, 0)) k
+ * with the bf16 value k the call writes (or would write) as its K output.
+ * k_rot has the layout of that K output; pos is documented per call. */
+typedef struct {
+    void *k_rot;                 /* bf16 destination; NULL = no rotation */
+    const float *pos;            /* fp32 (t, h, w) per token (4-byte aligned) */
+    int64_t pos_batch_stride;    /* elements between sessions in pos */
+    const double *t_origin_dev;  /* device fp64 added to every t, or NULL */
+    sr_rope_cfg cfg;             /* sub-blocks multiples of 8 summing to head_dim */
+    float out_scale;
+} sr_rope_out;
+
+/* Stream clock of a streaming session: *clock_dev += frames, on the stream
+ * (one-thread kernel, so that a step replayed from a CUDA graph sees the new
+ * value).  The clock is the t offset (sr_rope3d_apply's t_origin_dev) of the
+ * current chunk's first latent frame; a window slide of n frames advances it
+ * by n.  Defined by: "StreamRender-H3" (molayo1419.me), streaming context
+ * section (the fixed position template of the window; positions differ only
+ * by the step's shift, so each key is rotated once on entry).  clock_dev:
+ * 8-byte aligned device double. */
+int sr_stream_clock_advance(double *clock_dev, double frames, void *stream);
 
 /* ------------------------------------------------------------------------ */
 /* History-tier pooling.
@@ -141,6 +171,10 @@ int sr_qknorm_rope3d_apply(const void *x, void *y, void *y_raw, const float *gam
  *           pos_out + b*pos_batch_stride + 3*(f*cells + j); NULL = not written
  * slot_of_src int32 [n_frames*Gh*Gw] (device): slot_of_src[f*Gh*Gw + i] =
  *           f*cells + (cell of i); the same for every batch; NULL = not written
+ * rot       optional fused rotation of the pooled K (as rounded to bf16):
+ *           rot->k_rot has the strides of k_out; the position of pooled token
+ *           (b, f, j) is read at rot->pos + b*rot->pos_batch_stride + 3*(f*cells + j)
+ *           (the layout of pos_out).  NULL = none.
  * Input and output must not overlap.  head_dim in {64, 128};
  * pool_h, pool_w in [1, 8].
  */
@@ -157,7 +191,7 @@ int sr_history_compress(const void *k_in, const void *v_in, void *k_out, void *v
                         int64_t out_batch_stride, int64_t out_frame_stride,
                         int64_t out_token_stride, int64_t out_head_stride,
                         const float *frame_t, float *pos_out, int64_t pos_batch_stride,
-                        int32_t *slot_of_src, void *stream);
+                        int32_t *slot_of_src, const sr_rope_out *rot, void *stream);
 
 /* ------------------------------------------------------------------------ */
 /* KV append into the persistent window buffer.
@@ -176,6 +210,11 @@ int sr_history_compress(const void *k_in, const void *v_in, void *k_out, void *v
  * pos_src_batch_stride).  Bytes are copied exactly.
  * Any of k_src / v_src / pos_src may be NULL (that buffer is left alone).
  * n_valid_dev: optional int32[n_batch]; tokens n >= n_valid[b] are skipped.
+ * rot: optional fused rotation of K on its way in (the cache write and the
+ * RoPE in one pass): rot->k_rot is a buffer of k_buf's layout whose slots
+ * [dst_token, dst_token + n_tokens) receive the rotated K; the position of
+ * token n of session b is read at rot->pos + b*rot->pos_batch_stride + 3*n.
+ * With rot, k_buf may be NULL (only the rotated K is kept).  NULL = none.
  * Requires dst_token + n_tokens <= buf_tokens; head_dim in {64, 128}.
  */
 int sr_kv_append(void *k_buf, void *v_buf, float *pos_buf,
@@ -184,7 +223,7 @@ int sr_kv_append(void *k_buf, void *v_buf, float *pos_buf,
                  const void *k_src, const void *v_src, const float *pos_src,
                  int32_t n_tokens, const int32_t *n_valid_dev,
                  int64_t src_batch_stride, int64_t src_token_stride, int64_t src_head_stride,
-                 int64_t pos_src_batch_stride, void *stream);
+                 int64_t pos_src_batch_stride, const sr_rope_out *rot, void *stream);
 
 /* ------------------------------------------------------------------------ */
 /* Index gather / scatter of token rows (window partition and merge).
@@ -223,14 +262,17 @@ int sr_scatter_tokens(void *dst, const void *src, const int32_t *idx, int32_t n_
  *
  *   dst[b][s][h][:] = idx[b][s] >= 0 ? R(src_pos[idx[b][s]]) src[idx[b][s]][h][:] * out_scale : 0
  * Strides as for sr_gather_tokens; src_pos: fp32 [tokens][3] (t, h, w),
- * required.  cfg as for sr_rope3d_apply (sub-blocks multiples of 8 summing
+ * required; t_origin_dev: optional device fp64 added to every t (the
+ * absolute frame index of the call, so that the positions stay a fixed
+ * table), NULL = 0.  cfg as for sr_rope3d_apply (sub-blocks multiples of 8 summing
  * to head_dim).  head_dim in {64, 128}.  Returns SR_ERR_INVALID_ARG (nothing
  * launched) for bad sizes, strides, alignment or a missing src_pos.
  */
 int sr_gather_rope3d_tokens(void *dst, const void *src, const int32_t *idx, const float *src_pos, int32_t n_batch,
                             int32_t n_slots, int32_t n_heads, int32_t head_dim, sr_rope_cfg cfg, float out_scale,
                             int64_t src_token_stride, int64_t src_head_stride, int64_t dst_batch_stride,
-                            int64_t dst_slot_stride, int64_t dst_head_stride, void *stream);
+                            int64_t dst_slot_stride, int64_t dst_head_stride, const double *t_origin_dev,
+                            void *stream);
 
 /* ------------------------------------------------------------------------ */
 /* Fused chunk attention over [prompt | context | chunk] KV segments.
@@ -258,7 +300,9 @@ int sr_gather_rope3d_tokens(void *dst, const void *src, const int32_t *idx, cons
  * lse  fp32 [n_batch][n_heads][q_cap] natural-log LSE, or NULL
  * kv_len_dev int32 [n_batch][layout->n_seg] (device), 0 <= len <= cap
  * q_len_dev  int32 [n_batch] (device), 1 <= q_len <= q_cap; rows >= q_len are
- *      neither computed into o nor lse.
+ *      neither computed into o nor lse.  The host cannot check device values,
+ *      so the kernels clamp q_len to [0, q_cap]: an out-of-range value never
+ *      writes outside o or lse.
  * workspace  optional caller-owned device scratch of workspace_bytes >=
  *      sr_chunk_attention_workspace_bytes(n_batch, n_heads, head_dim, q_cap)
  *      bytes (16-byte aligned), or NULL.  With it, when the (session, head,
@@ -294,6 +338,23 @@ int sr_chunk_attention_fwd(const void *q, const void *k, const void *v, void *o,
  * only; reads the device's SM count (no allocation, no synchronisation). */
 size_t sr_chunk_attention_workspace_bytes(int32_t n_batch, int32_t n_heads, int32_t head_dim, int32_t q_cap);
 
+/* Bound of every pipeline wait inside the attention kernels, for the launches
+ * that follow on any thread (library-wide; default 1 s; 0 restores the
+ * default).  A wait that runs out raises SR_ERR_DEVICE_TIMEOUT in status_dev:
+ * the kernel then waits, again at most this long, for its own copies and
+ * tensor-core operations still in flight, releases its tensor memory and
+ * returns, leaving the context usable.  Not part of the method (the pages
+ * have no counterpart): the failure detection of this library. */
+int sr_set_wait_limit_ns(uint64_t limit_ns);
+
+/* Test hook of that failure path, not for production use (the pages have no
+ * counterpart): from the next attention launch on, the load of K tile `tile`
+ * (counted from each work item's first tile) is withheld, so the pipeline
+ * wait for it runs out after the limit above and the launch reports
+ * SR_ERR_DEVICE_TIMEOUT.  Nothing faults or hangs.  -1 (the default) turns it
+ * off; < -1 is rejected. */
+int sr_set_withheld_kv_tile(int32_t tile);
+
 /* Allocation-free variant of sr_chunk_attention_fwd (the pages have no
  * counterpart; this is a packaging option of this library).
  *
@@ -308,7 +369,10 @@ size_t sr_chunk_attention_workspace_bytes(int32_t n_batch, int32_t n_heads, int3
  * nothing and frees nothing.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address is looked up again when the
+ *     device's context has been re-created since (e.g. after
+ *     cudaDeviceReset), so the first call after such a reset must also come
+ *     before any capture.
  *   - Problems whose schedule needs more scratch than the array holds
  *     (sr_chunk_attention_workspace_bytes > SR_NOALLOC_SCRATCH_BYTES) are
  *     rejected with SR_ERR_UNSUPPORTED and nothing is launched.  On a 148-SM

@@ -48,28 +48,60 @@ class sr_kv_layout(ctypes.Structure):
     _fields_ = [("n_seg", ctypes.c_int32), ("cap", ctypes.c_int32 * SR_MAX_SEG)]
 
 
+class sr_rope_out(ctypes.Structure):
+    _fields_ = [("k_rot", ctypes.c_void_p), ("pos", ctypes.c_void_p), ("pos_batch_stride", ctypes.c_int64),
+                ("t_origin_dev", ctypes.c_void_p), ("cfg", sr_rope_cfg), ("out_scale", ctypes.c_float)]
+
+
+class RopeOut:
+    """A fused rotation of the K a call writes (sr_rope_out): k_rot is the
+    destination (the layout of the call's K output), pos the fp32 (t, h, w)
+    of every token ([B, N, 3], token stride 3), t_origin an optional CUDA
+    float64 tensor whose first element is added to every t."""
+
+    def __init__(self, k_rot: torch.Tensor, pos: torch.Tensor, split: Sequence[int], base: float = 10000.0,
+                 t_origin: Optional[torch.Tensor] = None, out_scale: float = 1.0):
+        self.k_rot, self.pos, self.split, self.base = k_rot, pos, split, base
+        self.t_origin, self.out_scale = t_origin, out_scale
+
+    def struct(self, n_tokens: int):
+        _cuda(self.k_rot, torch.bfloat16, "k_rot")
+        _cuda(self.pos, torch.float32, "rot.pos")
+        _cuda(self.t_origin, torch.float64, "t_origin")
+        B = self.pos.shape[0]
+        if tuple(self.pos.shape) != (B, n_tokens, 3) or self.pos.stride(1) != 3 or self.pos.stride(2) != 1:
+            raise ValueError(f"rotation positions must be [B, {n_tokens}, 3] with token stride 3")
+        cfg = sr_rope_cfg(float(self.base), int(self.split[0]), int(self.split[1]), int(self.split[2]))
+        return sr_rope_out(_ptr(self.k_rot), _ptr(self.pos), self.pos.stride(0), _ptr(self.t_origin), cfg,
+                           float(self.out_scale))
+
+
 _vp, _i32, _i64, _f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
 
 _SIGS = {
     "sr_version": ([], ctypes.c_int),
     "sr_get_last_error": ([], ctypes.c_char_p),
     "sr_rope3d_apply": ([_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, sr_rope_cfg, _f32,
-                         _i64, _i64, _i64, _i64, _i64, _i64, _i64, _vp], ctypes.c_int),
+                         _i64, _i64, _i64, _i64, _i64, _i64, _i64, _vp, _vp], ctypes.c_int),
     "sr_qknorm_rope3d_apply": ([_vp, _vp, _vp, _vp, _f32, _vp, _i32, _i32, _i32, _i32, _vp, sr_rope_cfg, _f32,
-                                _i64, _i64, _i64, _i64, _i64, _i64, _i64, _i64, _i64, _i64, _vp], ctypes.c_int),
+                                _i64, _i64, _i64, _i64, _i64, _i64, _i64, _i64, _i64, _i64, _vp, _vp],
+                               ctypes.c_int),
     "sr_gather_tokens": ([_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i64, _i64, _i64, _i64, _i64, _vp, _vp, _i64, _vp],
                          ctypes.c_int),
     "sr_scatter_tokens": ([_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i64, _i64, _i64, _i64, _i64, _vp], ctypes.c_int),
     "sr_gather_rope3d_tokens": ([_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, sr_rope_cfg, _f32,
-                                 _i64, _i64, _i64, _i64, _i64, _vp], ctypes.c_int),
+                                 _i64, _i64, _i64, _i64, _i64, _vp, _vp], ctypes.c_int),
     "sr_history_compress": ([_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, sr_pool_cfg,
-                             _i64, _i64, _i64, _i64, _i64, _i64, _i64, _i64, _vp, _vp, _i64, _vp, _vp],
-                            ctypes.c_int),
+                             _i64, _i64, _i64, _i64, _i64, _i64, _i64, _i64, _vp, _vp, _i64, _vp,
+                             ctypes.POINTER(sr_rope_out), _vp], ctypes.c_int),
     "sr_kv_append": ([_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _i32, _vp,
-                      _i64, _i64, _i64, _i64, _vp], ctypes.c_int),
+                      _i64, _i64, _i64, _i64, ctypes.POINTER(sr_rope_out), _vp], ctypes.c_int),
+    "sr_stream_clock_advance": ([_vp, ctypes.c_double, _vp], ctypes.c_int),
     "sr_chunk_attention_fwd": ([_vp, _vp, _vp, _vp, _vp, ctypes.POINTER(sr_kv_layout), _vp, _vp, _i32, _i32,
                                 _i32, _i32, _f32, _vp, ctypes.c_size_t, _vp, _vp], ctypes.c_int),
     "sr_chunk_attention_workspace_bytes": ([_i32, _i32, _i32, _i32], ctypes.c_size_t),
+    "sr_set_wait_limit_ns": ([ctypes.c_uint64], ctypes.c_int),
+    "sr_set_withheld_kv_tile": ([_i32], ctypes.c_int),
 }
 
 
@@ -127,9 +159,11 @@ def sr_version() -> int:
 
 def sr_rope3d_apply(x: torch.Tensor, y: torch.Tensor, pos: Optional[torch.Tensor], split: Sequence[int],
                     base: float = 10000.0, out_scale: float = 1.0, n_valid: Optional[torch.Tensor] = None,
-                    stream=None) -> None:
+                    t_origin: Optional[torch.Tensor] = None, stream=None) -> None:
     """x, y: [B, N, H, D] bf16 views (any strides, D contiguous); pos: [B, N, 3]
-    fp32 with token stride 3 (or None); n_valid: int32 [B] or None."""
+    fp32 with token stride 3 (or None); n_valid: int32 [B] or None; t_origin:
+    CUDA float64 tensor whose first element is added to every t (or None)."""
+    _cuda(t_origin, torch.float64, "t_origin")
     _cuda(x, torch.bfloat16, "x")
     _cuda(y, torch.bfloat16, "y")
     _cuda(pos, torch.float32, "pos")
@@ -145,15 +179,19 @@ def sr_rope3d_apply(x: torch.Tensor, y: torch.Tensor, pos: Optional[torch.Tensor
     cfg = sr_rope_cfg(float(base), int(split[0]), int(split[1]), int(split[2]))
     _check("sr_rope3d_apply", load().sr_rope3d_apply(
         _ptr(x), _ptr(y), _ptr(pos), B, N, H, D, _ptr(n_valid), cfg, float(out_scale),
-        x.stride(0), x.stride(1), x.stride(2), y.stride(0), y.stride(1), y.stride(2), pb, _stream(stream)))
+        x.stride(0), x.stride(1), x.stride(2), y.stride(0), y.stride(1), y.stride(2), pb, _ptr(t_origin),
+        _stream(stream)))
 
 
 def sr_qknorm_rope3d_apply(x: torch.Tensor, y: torch.Tensor, gamma: torch.Tensor, eps: float,
                            pos: Optional[torch.Tensor], split: Sequence[int], base: float = 10000.0,
                            out_scale: float = 1.0, n_valid: Optional[torch.Tensor] = None,
-                           y_raw: Optional[torch.Tensor] = None, stream=None) -> None:
+                           y_raw: Optional[torch.Tensor] = None, t_origin: Optional[torch.Tensor] = None,
+                           stream=None) -> None:
     """Per-head RMSNorm (gain gamma: fp32 [D], contiguous) then RoPE.  x, y,
-    y_raw: [B, N, H, D] bf16 views (D contiguous); pos as in sr_rope3d_apply."""
+    y_raw: [B, N, H, D] bf16 views (D contiguous); pos and t_origin as in
+    sr_rope3d_apply."""
+    _cuda(t_origin, torch.float64, "t_origin")
     _cuda(x, torch.bfloat16, "x")
     _cuda(y, torch.bfloat16, "y")
     _cuda(y_raw, torch.bfloat16, "y_raw")
@@ -177,7 +215,7 @@ def sr_qknorm_rope3d_apply(x: torch.Tensor, y: torch.Tensor, gamma: torch.Tensor
     _check("sr_qknorm_rope3d_apply", load().sr_qknorm_rope3d_apply(
         _ptr(x), _ptr(y), _ptr(y_raw), _ptr(gamma), float(eps), _ptr(pos), B, N, H, D, _ptr(n_valid), cfg,
         float(out_scale), x.stride(0), x.stride(1), x.stride(2), y.stride(0), y.stride(1), y.stride(2),
-        rs[0], rs[1], rs[2], pb, _stream(stream)))
+        rs[0], rs[1], rs[2], pb, _ptr(t_origin), _stream(stream)))
 
 
 def sr_gather_tokens(dst: torch.Tensor, src: torch.Tensor, idx: torch.Tensor, src_pos: Optional[torch.Tensor] = None,
@@ -206,9 +244,12 @@ def sr_gather_tokens(dst: torch.Tensor, src: torch.Tensor, idx: torch.Tensor, sr
 
 
 def sr_gather_rope3d_tokens(dst: torch.Tensor, src: torch.Tensor, idx: torch.Tensor, src_pos: torch.Tensor,
-                            split: Sequence[int], base: float = 10000.0, out_scale: float = 1.0, stream=None) -> None:
+                            split: Sequence[int], base: float = 10000.0, out_scale: float = 1.0,
+                            t_origin: Optional[torch.Tensor] = None, stream=None) -> None:
     """As sr_gather_tokens, every copied row rotated by the 3-D RoPE of its
-    source token's position src_pos [T, 3] (fp32, contiguous)."""
+    source token's position src_pos [T, 3] (fp32, contiguous), plus the first
+    element of t_origin (CUDA float64, optional) on t."""
+    _cuda(t_origin, torch.float64, "t_origin")
     for t, n in ((dst, "dst"), (src, "src")):
         _cuda(t, torch.bfloat16, n)
     _cuda(idx, torch.int32, "idx")
@@ -223,7 +264,7 @@ def sr_gather_rope3d_tokens(dst: torch.Tensor, src: torch.Tensor, idx: torch.Ten
     cfg = sr_rope_cfg(float(base), int(split[0]), int(split[1]), int(split[2]))
     _check("sr_gather_rope3d_tokens", load().sr_gather_rope3d_tokens(
         _ptr(dst), _ptr(src), _ptr(idx), _ptr(src_pos), B, S, H, D, cfg, float(out_scale), src.stride(0),
-        src.stride(1), dst.stride(0), dst.stride(1), dst.stride(2), _stream(stream)))
+        src.stride(1), dst.stride(0), dst.stride(1), dst.stride(2), _ptr(t_origin), _stream(stream)))
 
 
 def sr_scatter_tokens(dst: torch.Tensor, src: torch.Tensor, idx: torch.Tensor, stream=None) -> None:
@@ -246,11 +287,13 @@ def sr_history_compress(k_in: Optional[torch.Tensor], v_in: Optional[torch.Tenso
                         k_out: Optional[torch.Tensor], v_out: Optional[torch.Tensor],
                         grid_hw: Sequence[int], pool_hw: Sequence[int],
                         frame_t: Optional[torch.Tensor] = None, pos_out: Optional[torch.Tensor] = None,
-                        slot_of_src: Optional[torch.Tensor] = None, stream=None) -> None:
+                        slot_of_src: Optional[torch.Tensor] = None, rot: Optional[RopeOut] = None,
+                        stream=None) -> None:
     """k_in, v_in: [B, F, Gh*Gw, H, D] bf16 views; k_out, v_out: [B, F, cells, H, D]
     views (D contiguous; K and V views share strides); frame_t: fp32 [B, F]
     contiguous; pos_out: [B, F*cells, 3] fp32 (token stride 3); slot_of_src:
-    int32 [F*Gh*Gw]."""
+    int32 [F*Gh*Gw]; rot: fused rotation of the pooled K (rot.k_rot with
+    k_out's strides, rot.pos [B, F*cells, 3])."""
     ref_in = k_in if k_in is not None else v_in
     ref_out = k_out if k_out is not None else v_out
     for t, n in ((k_in, "k_in"), (v_in, "v_in"), (k_out, "k_out"), (v_out, "v_out")):
@@ -279,31 +322,39 @@ def sr_history_compress(k_in: Optional[torch.Tensor], v_in: Optional[torch.Tenso
         raise ValueError("slot_of_src must be int32 [F*Gh*Gw] contiguous")
     cfg = sr_pool_cfg(int(gh), int(gw), int(ph), int(pw))
     si, so = ref_in.stride(), ref_out.stride()
+    ro = None
+    if rot is not None:
+        if k_out is None or tuple(rot.k_rot.shape) != tuple(k_out.shape) or rot.k_rot.stride() != k_out.stride():
+            raise ValueError("rot.k_rot must have k_out's shape and strides")
+        ro = ctypes.byref(rot.struct(F * cells))
     _check("sr_history_compress", load().sr_history_compress(
         _ptr(k_in), _ptr(v_in), _ptr(k_out), _ptr(v_out), B, F, H, D, cfg,
         si[0], si[1], si[2], si[3], so[0], so[1], so[2], so[3],
-        _ptr(frame_t), _ptr(pos_out), pb, _ptr(slot_of_src), _stream(stream)))
+        _ptr(frame_t), _ptr(pos_out), pb, _ptr(slot_of_src), ro, _stream(stream)))
 
 
 def sr_kv_append(k_buf: Optional[torch.Tensor], v_buf: Optional[torch.Tensor], pos_buf: Optional[torch.Tensor],
                  dst_token: int, k_src: Optional[torch.Tensor], v_src: Optional[torch.Tensor],
-                 pos_src: Optional[torch.Tensor], n_valid: Optional[torch.Tensor] = None, stream=None) -> None:
+                 pos_src: Optional[torch.Tensor], n_valid: Optional[torch.Tensor] = None,
+                 rot: Optional[RopeOut] = None, stream=None) -> None:
     """k_buf, v_buf: [B, H, Cap, D] contiguous bf16; pos_buf: [B, Cap, 3] fp32
     contiguous; k_src, v_src: [B, N, H, D] views (D contiguous, same strides);
-    pos_src: [B, N, 3] (token stride 3)."""
+    pos_src: [B, N, 3] (token stride 3); rot: K rotated on its way into
+    rot.k_rot ([B, H, Cap, D] contiguous) at rot.pos [B, N, 3]; with rot,
+    k_buf may be None."""
     for t, n in ((k_buf, "k_buf"), (v_buf, "v_buf"), (k_src, "k_src"), (v_src, "v_src")):
         _cuda(t, torch.bfloat16, n)
     _cuda(pos_buf, torch.float32, "pos_buf")
     _cuda(pos_src, torch.float32, "pos_src")
     _cuda(n_valid, torch.int32, "n_valid")
-    buf = k_buf if k_buf is not None else v_buf
+    buf = k_buf if k_buf is not None else (v_buf if v_buf is not None else (rot.k_rot if rot is not None else None))
     src = k_src if k_src is not None else v_src
     if buf is None:
         raise ValueError("need a K or V buffer")
     B, H, cap, D = buf.shape
-    for t in (k_buf, v_buf):
+    for t in (k_buf, v_buf, rot.k_rot if rot is not None else None):
         if t is not None and (tuple(t.shape) != (B, H, cap, D) or not t.is_contiguous()):
-            raise ValueError("k_buf / v_buf must be contiguous [B, H, Cap, D]")
+            raise ValueError("k_buf / v_buf / rot.k_rot must be contiguous [B, H, Cap, D]")
     if pos_buf is not None and (tuple(pos_buf.shape) != (B, cap, 3) or not pos_buf.is_contiguous()):
         raise ValueError("pos_buf must be contiguous [B, Cap, 3]")
     if src is not None:
@@ -321,9 +372,16 @@ def sr_kv_append(k_buf: Optional[torch.Tensor], v_buf: Optional[torch.Tensor], p
         if tuple(pos_src.shape) != (B, N, 3) or pos_src.stride(1) != 3 or pos_src.stride(2) != 1:
             raise ValueError("pos_src must be [B, N, 3] with token stride 3")
         psb = pos_src.stride(0)
+    ro = ctypes.byref(rot.struct(N)) if rot is not None else None
     _check("sr_kv_append", load().sr_kv_append(
         _ptr(k_buf), _ptr(v_buf), _ptr(pos_buf), B, H, D, cap, int(dst_token), _ptr(k_src), _ptr(v_src),
-        _ptr(pos_src), N, _ptr(n_valid), ss[0], ss[1], ss[2], psb, _stream(stream)))
+        _ptr(pos_src), N, _ptr(n_valid), ss[0], ss[1], ss[2], psb, ro, _stream(stream)))
+
+
+def sr_stream_clock_advance(clock: torch.Tensor, frames: float, stream=None) -> None:
+    """clock: CUDA float64 tensor; its first element += frames, on the stream."""
+    _cuda(clock, torch.float64, "clock")
+    _check("sr_stream_clock_advance", load().sr_stream_clock_advance(_ptr(clock), float(frames), _stream(stream)))
 
 
 def make_layout(caps: Sequence[int]) -> sr_kv_layout:
@@ -334,6 +392,17 @@ def make_layout(caps: Sequence[int]) -> sr_kv_layout:
     for i, c in enumerate(caps):
         lay.cap[i] = int(c)
     return lay
+
+
+def sr_set_wait_limit_ns(limit_ns: int) -> None:
+    """Bound of every pipeline wait in the attention kernels (0: the 1 s default)."""
+    _check("sr_set_wait_limit_ns", load().sr_set_wait_limit_ns(int(limit_ns)))
+
+
+def sr_set_withheld_kv_tile(tile: int) -> None:
+    """Test hook of the bounded-wait failure path: withhold the load of one K
+    tile in later attention launches (-1: off)."""
+    _check("sr_set_withheld_kv_tile", load().sr_set_withheld_kv_tile(int(tile)))
 
 
 def sr_chunk_attention_workspace_bytes(n_batch: int, n_heads: int, head_dim: int, q_cap: int) -> int:

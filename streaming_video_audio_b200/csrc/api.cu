@@ -72,7 +72,8 @@ const char *sr_get_last_error(void) { return g_last_error; }
 int sr_rope3d_apply(const void *x, void *y, const float *pos, int32_t n_batch, int32_t n_tokens, int32_t n_heads,
                     int32_t head_dim, const int32_t *n_valid_dev, sr_rope_cfg cfg, float out_scale,
                     int64_t x_batch_stride, int64_t x_token_stride, int64_t x_head_stride, int64_t y_batch_stride,
-                    int64_t y_token_stride, int64_t y_head_stride, int64_t pos_batch_stride, void *stream) {
+                    int64_t y_token_stride, int64_t y_head_stride, int64_t pos_batch_stride,
+                    const double *t_origin_dev, void *stream) {
     g_last_error[0] = 0;
     if (n_batch < 0 || n_tokens < 0 || n_heads < 1 || n_batch > 65535)
         return set_error(SR_ERR_INVALID_ARG, "rope3d: bad sizes (batch %d, tokens %d, heads %d)", n_batch,
@@ -92,9 +93,12 @@ int sr_rope3d_apply(const void *x, void *y, const float *pos, int32_t n_batch, i
         return set_error(SR_ERR_INVALID_ARG, "rope3d: strides must be multiples of 8 elements");
     if (pos && (reinterpret_cast<uintptr_t>(pos) & 3u))
         return set_error(SR_ERR_INVALID_ARG, "rope3d: pos must be 4-byte aligned");
+    if (t_origin_dev && (reinterpret_cast<uintptr_t>(t_origin_dev) & 7u))
+        return set_error(SR_ERR_INVALID_ARG, "rope3d: t_origin must be 8-byte aligned");
     RopeLaunch l{x, y, pos, n_valid_dev, n_batch, n_tokens, n_heads, head_dim, cfg, out_scale,
                  x_batch_stride, x_token_stride, x_head_stride, y_batch_stride, y_token_stride, y_head_stride,
                  pos_batch_stride, static_cast<cudaStream_t>(stream)};
+    l.t_origin = t_origin_dev;
     return launch_rope3d(l);
 }
 
@@ -104,7 +108,7 @@ int sr_qknorm_rope3d_apply(const void *x, void *y, void *y_raw, const float *gam
                            int64_t x_token_stride, int64_t x_head_stride, int64_t y_batch_stride,
                            int64_t y_token_stride, int64_t y_head_stride, int64_t yraw_batch_stride,
                            int64_t yraw_token_stride, int64_t yraw_head_stride, int64_t pos_batch_stride,
-                           void *stream) {
+                           const double *t_origin_dev, void *stream) {
     g_last_error[0] = 0;
     if (!gamma) return set_error(SR_ERR_INVALID_ARG, "qknorm_rope3d: gamma is NULL");
     if (reinterpret_cast<uintptr_t>(gamma) & 15u)
@@ -139,6 +143,9 @@ int sr_qknorm_rope3d_apply(const void *x, void *y, void *y_raw, const float *gam
     RopeLaunch l{x, y, pos, n_valid_dev, n_batch, n_tokens, n_heads, head_dim, cfg, out_scale,
                  x_batch_stride, x_token_stride, x_head_stride, y_batch_stride, y_token_stride, y_head_stride,
                  pos_batch_stride, static_cast<cudaStream_t>(stream)};
+    if (t_origin_dev && (reinterpret_cast<uintptr_t>(t_origin_dev) & 7u))
+        return set_error(SR_ERR_INVALID_ARG, "qknorm_rope3d: t_origin must be 8-byte aligned");
+    l.t_origin = t_origin_dev;
     l.gamma = gamma;
     l.eps = eps;
     l.y_raw = y_raw;
@@ -146,6 +153,23 @@ int sr_qknorm_rope3d_apply(const void *x, void *y, void *y_raw, const float *gam
     l.rt = yraw_token_stride;
     l.rh = yraw_head_stride;
     return launch_rope3d(l);
+}
+
+// Checks of an optional fused rotation (sr_rope_out) of a call whose K
+// output has head_dim elements per row.
+static int rope_out_check(const char *name, const sr_rope_out *rot, int32_t head_dim) {
+    if (!rot || !rot->k_rot) return SR_OK;
+    const sr_rope_cfg &c = rot->cfg;
+    if (c.d_t < 0 || c.d_h < 0 || c.d_w < 0 || c.d_t % 8 || c.d_h % 8 || c.d_w % 8 || c.d_t + c.d_h + c.d_w != head_dim)
+        return set_error(SR_ERR_INVALID_ARG, "%s: rotation sub-blocks %d/%d/%d must be multiples of 8 summing to %d",
+                         name, c.d_t, c.d_h, c.d_w, head_dim);
+    if (!(c.base > 0.f)) return set_error(SR_ERR_INVALID_ARG, "%s: rotation base must be positive", name);
+    if (!aligned16(rot->k_rot)) return set_error(SR_ERR_INVALID_ARG, "%s: k_rot must be 16-byte aligned", name);
+    if (!rot->pos || (reinterpret_cast<uintptr_t>(rot->pos) & 3u))
+        return set_error(SR_ERR_INVALID_ARG, "%s: the rotation needs positions (4-byte aligned)", name);
+    if (rot->t_origin_dev && (reinterpret_cast<uintptr_t>(rot->t_origin_dev) & 7u))
+        return set_error(SR_ERR_INVALID_ARG, "%s: t_origin must be 8-byte aligned", name);
+    return SR_OK;
 }
 
 static int gather_common(const char *name, void *dst, const void *src, const int32_t *idx, int32_t n_batch,
@@ -211,7 +235,8 @@ int sr_scatter_tokens(void *dst, const void *src, const int32_t *idx, int32_t n_
 int sr_gather_rope3d_tokens(void *dst, const void *src, const int32_t *idx, const float *src_pos, int32_t n_batch,
                             int32_t n_slots, int32_t n_heads, int32_t head_dim, sr_rope_cfg cfg, float out_scale,
                             int64_t src_token_stride, int64_t src_head_stride, int64_t dst_batch_stride,
-                            int64_t dst_slot_stride, int64_t dst_head_stride, void *stream) {
+                            int64_t dst_slot_stride, int64_t dst_head_stride, const double *t_origin_dev,
+                            void *stream) {
     g_last_error[0] = 0;
     GatherLaunch l{};
     int rc = gather_common("gather_rope3d_tokens", dst, src, idx, n_batch, n_slots, n_heads, head_dim,
@@ -228,9 +253,12 @@ int sr_gather_rope3d_tokens(void *dst, const void *src, const int32_t *idx, cons
     l.src = src;
     l.src_pos = src_pos;
     l.scatter = false;
+    if (t_origin_dev && (reinterpret_cast<uintptr_t>(t_origin_dev) & 7u))
+        return set_error(SR_ERR_INVALID_ARG, "gather_rope3d_tokens: t_origin must be 8-byte aligned");
     l.rope = true;
     l.cfg = cfg;
     l.out_scale = out_scale;
+    l.t_origin = t_origin_dev;
     l.stream = static_cast<cudaStream_t>(stream);
     return launch_gather(l);
 }
@@ -240,7 +268,7 @@ int sr_history_compress(const void *k_in, const void *v_in, void *k_out, void *v
                         int64_t in_frame_stride, int64_t in_token_stride, int64_t in_head_stride,
                         int64_t out_batch_stride, int64_t out_frame_stride, int64_t out_token_stride,
                         int64_t out_head_stride, const float *frame_t, float *pos_out, int64_t pos_batch_stride,
-                        int32_t *slot_of_src, void *stream) {
+                        int32_t *slot_of_src, const sr_rope_out *rot, void *stream) {
     g_last_error[0] = 0;
     if (n_batch < 0 || n_frames < 0 || n_heads < 1)
         return set_error(SR_ERR_INVALID_ARG, "history_compress: bad sizes");
@@ -257,17 +285,28 @@ int sr_history_compress(const void *k_in, const void *v_in, void *k_out, void *v
                       out_frame_stride, out_token_stride, out_head_stride})
         if (!stride_ok(s)) return set_error(SR_ERR_INVALID_ARG, "history_compress: strides must be multiples of 8");
     if (pos_out && !frame_t) return set_error(SR_ERR_INVALID_ARG, "history_compress: pos_out needs frame_t");
+    int rc = rope_out_check("history_compress", rot, head_dim);
+    if (rc != SR_OK) return rc;
+    if (rot && rot->k_rot && !k_in) return set_error(SR_ERR_INVALID_ARG, "history_compress: rotation needs K");
     PoolLaunch l{k_in, v_in, k_out, v_out, n_batch, n_frames, n_heads, head_dim, cfg,
                  in_batch_stride, in_frame_stride, in_token_stride, in_head_stride,
                  out_batch_stride, out_frame_stride, out_token_stride, out_head_stride,
                  frame_t, pos_out, pos_batch_stride, slot_of_src, static_cast<cudaStream_t>(stream)};
+    if (rot && rot->k_rot) {
+        l.k_rot = rot->k_rot;
+        l.rot_pos = rot->pos;
+        l.rot_pos_b = rot->pos_batch_stride;
+        l.t_origin = rot->t_origin_dev;
+        l.rot_cfg = rot->cfg;
+        l.rot_scale = rot->out_scale;
+    }
     return launch_history_compress(l);
 }
 
 int sr_kv_append(void *k_buf, void *v_buf, float *pos_buf, int32_t n_batch, int32_t n_heads, int32_t head_dim,
                  int32_t buf_tokens, int32_t dst_token, const void *k_src, const void *v_src, const float *pos_src,
                  int32_t n_tokens, const int32_t *n_valid_dev, int64_t src_batch_stride, int64_t src_token_stride,
-                 int64_t src_head_stride, int64_t pos_src_batch_stride, void *stream) {
+                 int64_t src_head_stride, int64_t pos_src_batch_stride, const sr_rope_out *rot, void *stream) {
     g_last_error[0] = 0;
     if (n_batch < 0 || n_heads < 1 || n_tokens < 0 || buf_tokens < 0 || dst_token < 0)
         return set_error(SR_ERR_INVALID_ARG, "kv_append: bad sizes");
@@ -276,8 +315,12 @@ int sr_kv_append(void *k_buf, void *v_buf, float *pos_buf, int32_t n_batch, int3
         return set_error(SR_ERR_INVALID_ARG, "kv_append: slots [%d, %d) exceed the buffer (%d tokens)", dst_token,
                          dst_token + n_tokens, buf_tokens);
     if (n_batch == 0 || n_tokens == 0) return SR_OK;
-    if ((k_src && !k_buf) || (v_src && !v_buf) || (pos_src && !pos_buf))
+    const bool rotate = rot && rot->k_rot;
+    if ((k_src && !k_buf && !rotate) || (v_src && !v_buf) || (pos_src && !pos_buf))
         return set_error(SR_ERR_INVALID_ARG, "kv_append: source given without its buffer");
+    int rc = rope_out_check("kv_append", rot, head_dim);
+    if (rc != SR_OK) return rc;
+    if (rotate && !k_src) return set_error(SR_ERR_INVALID_ARG, "kv_append: rotation needs k_src");
     for (const void *p : {static_cast<const void *>(k_buf), static_cast<const void *>(v_buf), k_src, v_src})
         if (p && !aligned16(p)) return set_error(SR_ERR_INVALID_ARG, "kv_append: tensors must be 16-byte aligned");
     if (!stride_ok(src_batch_stride) || !stride_ok(src_token_stride) || !stride_ok(src_head_stride))
@@ -285,12 +328,28 @@ int sr_kv_append(void *k_buf, void *v_buf, float *pos_buf, int32_t n_batch, int3
     AppendLaunch l{k_buf, v_buf, pos_buf, n_batch, n_heads, head_dim, buf_tokens, dst_token, k_src, v_src, pos_src,
                    n_tokens, n_valid_dev, src_batch_stride, src_token_stride, src_head_stride, pos_src_batch_stride,
                    static_cast<cudaStream_t>(stream)};
+    if (rotate) {
+        if (n_batch > 65535) return set_error(SR_ERR_INVALID_ARG, "kv_append: too many sessions");
+        l.k_rot = rot->k_rot;
+        l.rot_pos = rot->pos;
+        l.rot_pos_b = rot->pos_batch_stride;
+        l.t_origin = rot->t_origin_dev;
+        l.rot_cfg = rot->cfg;
+        l.rot_scale = rot->out_scale;
+    }
     return launch_kv_append(l);
+}
+
+int sr_stream_clock_advance(double *clock_dev, double frames, void *stream) {
+    g_last_error[0] = 0;
+    if (!clock_dev || (reinterpret_cast<uintptr_t>(clock_dev) & 7u))
+        return set_error(SR_ERR_INVALID_ARG, "stream_clock_advance: clock must be an 8-byte aligned device double");
+    return launch_clock_advance(clock_dev, frames, static_cast<cudaStream_t>(stream));
 }
 
 size_t sr_chunk_attention_workspace_bytes(int32_t n_batch, int32_t n_heads, int32_t head_dim, int32_t q_cap) {
     if (n_batch < 1 || n_heads < 1 || q_cap < 1 || (head_dim != 64 && head_dim != 128)) return 0;
-    return attention_schedule(n_batch, n_heads, head_dim, q_cap, attention_sm_count()).workspace_bytes;
+    return attention_schedule(n_batch, n_heads, head_dim, q_cap, attention_slots(head_dim)).workspace_bytes;
 }
 
 int sr_chunk_attention_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
@@ -342,6 +401,8 @@ int sr_chunk_attention_fwd(const void *q, const void *k, const void *v, void *o,
     a.workspace = workspace;
     a.workspace_bytes = workspace ? workspace_bytes : 0;
     a.stream = static_cast<cudaStream_t>(stream);
+    a.wait_limit_ns = attention_wait_limit_ns();
+    a.withheld_tile = attention_withheld_tile();
     return launch_chunk_attention(a);
 }
 

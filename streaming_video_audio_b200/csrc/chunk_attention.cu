@@ -1,5 +1,8 @@
 // chunk_attention.cu -- fused chunk attention over [prompt | context | chunk]
-// KV segments on sm_100a (tcgen05 tensor cores, TMEM accumulators, TMA).
+// KV segments on sm_100a (tcgen05 tensor cores, TMEM accumulators, TMA): the
+// dispatch of sr_chunk_attention_fwd, the split-KV work list and merge, and
+// the single-SM kernel used at head_dim 64 (head_dim 128 runs on CTA pairs,
+// pair_attention.cu).
 //
 // What it computes (plain definition, no causal mask): for every valid query
 // row i of a (session, head),
@@ -37,6 +40,7 @@
 // aliases the first 64 columns of S_t.  Every wait is bounded
 // (sr_device.cuh): a stuck pipeline sets the status word and the CTA returns
 // instead of hanging.
+#include <atomic>
 #include <mutex>
 
 #include <cuda.h>
@@ -87,6 +91,8 @@ struct AttnParams {
     int32_t split;
     float *ws_o;             // [slot][2][128][D] unnormalised partial O (log2-domain max m, sum l)
     float *ws_ml;            // [slot][m | l][2][128]
+    uint64_t wait_limit_ns;
+    int32_t withheld_tile;   // test hook: the K tile whose load is withheld (-1: none)
 };
 
 template <int D>
@@ -98,8 +104,8 @@ struct Smem {
     static constexpr int kV = kK + kStages * kTileBytes;
     static constexpr int kBar = kV + kStages * kTileBytes;
     // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S],
-    // s_full[2], p_full[2], o_done[2], stats_ready[2]
-    static constexpr int kNumBars = 1 + 4 * kStages + 4 * kQTiles;
+    // s_full[2], p_full[2], o_done[2], stats_ready[2], drain
+    static constexpr int kNumBars = 1 + 4 * kStages + 4 * kQTiles + 1;
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kRow = kMisc + 16 + 12 * SR_MAX_SEG + 16;   // float l[2][128], m[2][128]
     static constexpr int kEnd = kRow + 2 * kQTiles * kTileM * 4;
@@ -121,8 +127,8 @@ struct TileWalk {
 
 
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                          int32_t *status) {
-    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, status));
+                                          int32_t *status, uint64_t limit) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, status, limit));
 }
 
 template <int D>
@@ -146,7 +152,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int qb = unit % p.qb_per_head;
     const int bh = unit / p.qb_per_head;
     const int h = bh % p.n_heads, b = bh / p.n_heads;
-    const int q_len = p.q_len[b];
+    // q_len is caller data on the device: clamped to [0, q_cap] so that no
+    // row past the o / lse buffers is ever written, whatever it holds
+    const int q_len = min(max(p.q_len[b], 0), p.q_cap);
     const int q0 = qb * kQTiles * kTileM;
     if (q0 >= q_len) return;   // uniform for the whole CTA
 
@@ -160,6 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *p_full = s_full + kQTiles;         // [2] softmax t -> MMA (P_t written, O_t rescaled)
     uint64_t *o_done = p_full + kQTiles;         // [2] MMA (PV_t) -> epilogue
     uint64_t *stats_ready = o_done + kQTiles;    // [2] softmax t -> epilogue: final row max / sum
+    uint64_t *drain = stats_ready + kQTiles;     // every MMA issued so far is complete
     // Every waiter consumes each phase of its barrier in order, so parity
     // waits never alias: a barrier is never more than one phase ahead of the
     // phase its waiter asks for.
@@ -189,6 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&o_done[t], 1);
             mbar_init(&stats_ready[t], 4);
         }
+        mbar_init(drain, 1);
         *abort_flag = 0;
         int total = 0;
 #pragma unroll
@@ -224,6 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int n_tiles = *n_tiles_s;
     const int n_seg = p.n_seg;
     const float sl2 = p.scale_log2;
+    const uint64_t limit = p.wait_limit_ns;
 
     if (warp < 4 * kQTiles) {
         // ================================================================ softmax of tile t
@@ -240,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         w.t = walk_start[1];
         for (int j = 0; j < n_tiles; ++j, w.next(seg_ntile, n_seg)) {
             const int valid = min(kTileN, seg_len[w.s] - w.t * kTileN);
-            if (!(ok = warp_wait(&s_full[t], j & 1, abort_flag, p.status))) break;
+            if (!(ok = warp_wait(&s_full[t], j & 1, abort_flag, p.status, limit))) break;
             tc_fence_after();
             float s[kTileN];
             {
@@ -333,8 +344,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     continue;
                 }
                 if (!ok) break;
-                if (!(ok = warp_wait(&stats_ready[t], 0, abort_flag, p.status))) break;
-                if (!(ok = warp_wait(&o_done[t], (n_tiles - 1) & 1, abort_flag, p.status))) break;
+                if (!(ok = warp_wait(&stats_ready[t], 0, abort_flag, p.status, limit))) break;
+                if (!(ok = warp_wait(&o_done[t], (n_tiles - 1) & 1, abort_flag, p.status, limit))) break;
                 tc_fence_after();
                 const float l_row = row_l[t * kTileM + row];
                 const float inv_l = 1.0f / l_row;
@@ -371,8 +382,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float m_part = -INFINITY, l_part = 0.f;
                 if (n_tiles > 0) {
                     if (!ok) break;
-                    if (!(ok = warp_wait(&stats_ready[t], 0, abort_flag, p.status))) break;
-                    if (!(ok = warp_wait(&o_done[t], (n_tiles - 1) & 1, abort_flag, p.status))) break;
+                    if (!(ok = warp_wait(&stats_ready[t], 0, abort_flag, p.status, limit))) break;
+                    if (!(ok = warp_wait(&o_done[t], (n_tiles - 1) & 1, abort_flag, p.status, limit))) break;
                     tc_fence_after();
                     m_part = row_m[t * kTileM + row];
                     l_part = row_l[t * kTileM + row];
@@ -407,6 +418,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int pn = 0; pn < L::kPanels; ++pn)
                         tma_load_3d(smem + L::kQ + t * L::kTileBytes + pn * kPanelBytes, &tmQ, pn * 64,
                                     q0 + t * kTileM, bh, q_full);
+                int k_last[kStages], v_last[kStages];   // last tile loaded into each stage (for the drain)
+#pragma unroll
+                for (int i = 0; i < kStages; ++i) k_last[i] = v_last[i] = -1;
                 TileWalk w;
                 w.s = walk_start[0];
                 w.t = walk_start[1];
@@ -414,18 +428,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int st = j % kStages;
                     const uint32_t ph = (j / kStages) & 1;
                     const int row0 = seg_start[w.s] + w.t * kTileN;
-                    if (!mbar_wait(&k_empty[st], ph ^ 1, abort_flag, p.status)) break;
-                    mbar_expect_tx(&k_full[st], L::kTileBytes);
+                    if (!mbar_wait(&k_empty[st], ph ^ 1, abort_flag, p.status, limit)) break;
+                    if (j != p.withheld_tile) {
+                        mbar_expect_tx(&k_full[st], L::kTileBytes);
 #pragma unroll
-                    for (int pn = 0; pn < L::kPanels; ++pn)
-                        tma_load_3d(smem + L::kK + st * L::kTileBytes + pn * kPanelBytes, &tmK, pn * 64, row0, bh,
-                                    &k_full[st]);
-                    if (!mbar_wait(&v_empty[st], ph ^ 1, abort_flag, p.status)) break;
+                        for (int pn = 0; pn < L::kPanels; ++pn)
+                            tma_load_3d(smem + L::kK + st * L::kTileBytes + pn * kPanelBytes, &tmK, pn * 64, row0, bh,
+                                        &k_full[st]);
+                        k_last[st] = j;
+                    }
+                    if (!mbar_wait(&v_empty[st], ph ^ 1, abort_flag, p.status, limit)) break;
                     mbar_expect_tx(&v_full[st], L::kTileBytes);
 #pragma unroll
                     for (int pn = 0; pn < L::kPanels; ++pn)
                         tma_load_3d(smem + L::kV + st * L::kTileBytes + pn * kPanelBytes, &tmV, pn * 64, row0, bh,
                                     &v_full[st]);
+                    v_last[st] = j;
+                }
+                if (*abort_flag) {
+                    // wait, bounded, for the loads still in flight into this CTA
+                    mbar_drain(q_full, 0, limit);
+                    for (int i = 0; i < kStages; ++i) {
+                        if (k_last[i] >= 0) mbar_drain(&k_full[i], (k_last[i] / kStages) & 1, limit);
+                        if (v_last[i] >= 0) mbar_drain(&v_full[i], (v_last[i] / kStages) & 1, limit);
+                    }
                 }
             }
         } else if (warp == kWarpMma) {
@@ -462,7 +488,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                      (acc || kk > 0) ? 1u : 0u);
                     umma_commit(&o_done[t]);
                 };
-                bool ok = mbar_wait(q_full, 0, abort_flag, p.status) && mbar_wait(&k_full[0], 0, abort_flag, p.status);
+                bool ok = mbar_wait(q_full, 0, abort_flag, p.status, limit) &&
+                          mbar_wait(&k_full[0], 0, abort_flag, p.status, limit);
                 if (ok) {
                     tc_fence_after();
                     issue_qk(0, 0);
@@ -473,16 +500,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int st = j % kStages;
                     const int st1 = (j + 1) % kStages;
                     const bool more = j + 1 < n_tiles;
-                    if (!(ok = mbar_wait(&v_full[st], (j / kStages) & 1, abort_flag, p.status))) break;
-                    if (!(ok = mbar_wait(&p_full[0], j & 1, abort_flag, p.status))) break;
+                    if (!(ok = mbar_wait(&v_full[st], (j / kStages) & 1, abort_flag, p.status, limit))) break;
+                    if (!(ok = mbar_wait(&p_full[0], j & 1, abort_flag, p.status, limit))) break;
                     tc_fence_after();
                     issue_pv(0, st, j > 0);
                     if (more) {
-                        if (!(ok = mbar_wait(&k_full[st1], ((j + 1) / kStages) & 1, abort_flag, p.status))) break;
+                        if (!(ok = mbar_wait(&k_full[st1], ((j + 1) / kStages) & 1, abort_flag, p.status, limit))) break;
                         tc_fence_after();
                         issue_qk(0, st1);
                     }
-                    if (!(ok = mbar_wait(&p_full[1], j & 1, abort_flag, p.status))) break;
+                    if (!(ok = mbar_wait(&p_full[1], j & 1, abort_flag, p.status, limit))) break;
                     tc_fence_after();
                     issue_pv(1, st, j > 0);
                     umma_commit(&v_empty[st]);
@@ -491,6 +518,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         umma_commit(&k_empty[st1]);
                     }
                 }
+                // every MMA issued so far complete before the tensor and shared
+                // memory may be released (matters after an abort)
+                umma_commit(drain);
+                mbar_drain(drain, 0, limit);
             }
         }
     }
@@ -530,7 +561,7 @@ __global__ void __launch_bounds__(256) split_combine_kernel(const CombineParams 
     const int qb = unit % c.qb_per_head, bh = unit / c.qb_per_head;
     const int h = bh % c.n_heads, b = bh / c.n_heads;
     const int grow = qb * kQTiles * kTileM + r2;
-    if (grow >= c.q_len[b]) return;
+    if (grow >= min(max(c.q_len[b], 0), c.q_cap)) return;   // clamped as in the attention kernel
     float mmax = -INFINITY;
     for (int q = 0; q < c.split; ++q)
         mmax = fmaxf(mmax, c.ws_ml[static_cast<size_t>(tail * c.split + q) * 4 * kTileM + t * kTileM + row]);
@@ -597,6 +628,8 @@ int launch(const AttnLaunch &a) {
     p.n_heads = a.n_heads;
     p.q_cap = a.q_cap;
     p.scale_log2 = static_cast<float>(static_cast<double>(a.softmax_scale) * 1.4426950408889634);
+    p.wait_limit_ns = a.wait_limit_ns;
+    p.withheld_tile = a.withheld_tile;
     const AttnSchedule sc = attention_schedule(a.n_batch, a.n_heads, D, a.q_cap, sm_count());
     p.qb_per_head = sc.qb_per_head;
     p.n_full = sc.n_full;
@@ -624,18 +657,34 @@ int launch(const AttnLaunch &a) {
     chunk_attention_kernel<D><<<static_cast<unsigned>(items), kThreads, L::kAlloc, a.stream>>>(tq, tk, tv, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return set_cuda_error("chunk_attention launch", e);
-    if (p.split > 1) {
-        CombineParams c{p.ws_o, p.ws_ml, p.o, p.lse, p.q_len, p.n_full, p.split, sc.tail_units, p.qb_per_head,
-                        p.n_heads, p.q_cap};
-        const int64_t threads = static_cast<int64_t>(sc.tail_units) * kQTiles * kTileM * (D / 8);
-        split_combine_kernel<D><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, a.stream>>>(c);
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return set_cuda_error("split_combine launch", e);
-    }
+    if (p.split > 1)
+        return launch_split_combine(p.ws_o, p.ws_ml, p.o, p.lse, p.q_len, p.n_full, p.split, sc.tail_units,
+                                    p.qb_per_head, p.n_heads, p.q_cap, D, a.stream);
     return SR_OK;
 }
 
+std::atomic<uint64_t> g_wait_limit_ns{kWaitLimitNs};
+std::atomic<int32_t> g_withheld_tile{-1};
+
 }  // namespace
+
+uint64_t attention_wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
+int32_t attention_withheld_tile() { return g_withheld_tile.load(std::memory_order_relaxed); }
+
+int launch_split_combine(const float *ws_o, const float *ws_ml, void *o, float *lse, const int32_t *q_len,
+                         int32_t n_full, int32_t split, int32_t tail_units, int32_t qb_per_head, int32_t n_heads,
+                         int32_t q_cap, int32_t head_dim, cudaStream_t stream) {
+    CombineParams c{ws_o, ws_ml, static_cast<__nv_bfloat16 *>(o), lse, q_len, n_full, split, tail_units,
+                    qb_per_head, n_heads, q_cap};
+    const int64_t threads = static_cast<int64_t>(tail_units) * kQTiles * kTileM * (head_dim / 8);
+    const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+    if (head_dim == 128)
+        split_combine_kernel<128><<<blocks, 256, 0, stream>>>(c);
+    else
+        split_combine_kernel<64><<<blocks, 256, 0, stream>>>(c);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SR_OK : set_cuda_error("split_combine launch", e);
+}
 
 AttnSchedule attention_schedule(int32_t n_batch, int32_t n_heads, int32_t head_dim, int32_t q_cap, int32_t sms) {
     AttnSchedule sc{};
@@ -664,8 +713,11 @@ AttnSchedule attention_schedule(int32_t n_batch, int32_t n_heads, int32_t head_d
 
 int attention_sm_count() { return sm_count(); }
 
+int attention_slots(int32_t head_dim) { return head_dim == 128 ? attention_pair_slots() : sm_count(); }
+
 int launch_chunk_attention(const AttnLaunch &a) {
-    if (a.head_dim == 128) return launch<128>(a);
+    if (a.head_dim == 128)
+        return launch_pair_attention(a, attention_schedule(a.n_batch, a.n_heads, 128, a.q_cap, attention_pair_slots()));
     if (a.head_dim == 64) return launch<64>(a);
     return set_error(SR_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
 }
@@ -689,23 +741,56 @@ namespace {
 static __device__ __align__(256) uint8_t g_noalloc_scratch[SR_NOALLOC_SCRATCH_BYTES];
 
 std::mutex g_noalloc_mutex;
-void *g_noalloc_ptr[64] = {};   // device address of g_noalloc_scratch, per device
+void *g_noalloc_ptr[64] = {};                  // device address of g_noalloc_scratch, per device
+unsigned long long g_noalloc_ctx[64] = {};     // id of the context that address belongs to
+
+// Unique id of the calling thread's current CUDA context (0 if there is none
+// yet, or the driver does not offer the query).  Ids are never reused within
+// a process, so a changed id means the device's context was re-created (for
+// instance after cudaDeviceReset) and the module, with its static array, was
+// loaded again at a possibly different address.
+unsigned long long current_context_id() {
+    using GetCurrentFn = CUresult (*)(CUcontext *);
+    using GetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+    static std::once_flag once;
+    static GetCurrentFn get_current = nullptr;
+    static GetIdFn get_id = nullptr;
+    std::call_once(once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrentFn>(fn);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetIdFn>(fn);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
 
 // Device address of the scratch array on the current device.  The host-side
 // name g_noalloc_scratch is only a stand-in for the symbol; the address a
-// kernel may use comes from cudaGetSymbolAddress, resolved once per device
-// with that device current.
+// kernel may use comes from cudaGetSymbolAddress, resolved with that device
+// current the first time a device is used, and again whenever the device's
+// context has changed since (the cached address would point into a module
+// that no longer exists).
 int noalloc_scratch(void **out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return set_cuda_error("cudaGetDevice", e);
     if (dev < 0 || dev >= 64) return set_error(SR_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
     std::lock_guard<std::mutex> guard(g_noalloc_mutex);
-    if (!g_noalloc_ptr[dev]) {
+    const unsigned long long ctx = current_context_id();
+    if (!g_noalloc_ptr[dev] || ctx == 0 || ctx != g_noalloc_ctx[dev]) {
         void *ptr = nullptr;
         e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
         if (e != cudaSuccess) return set_cuda_error("cudaGetSymbolAddress(static attention scratch)", e);
         g_noalloc_ptr[dev] = ptr;
+        g_noalloc_ctx[dev] = current_context_id();   // the lookup itself may have created the context
     }
     *out = g_noalloc_ptr[dev];
     return SR_OK;
@@ -731,4 +816,15 @@ extern "C" int sr_chunk_attention_fwd_noalloc(const void *q, const void *k, cons
     if (rc != SR_OK) return rc;
     return sr_chunk_attention_fwd(q, k, v, o, lse, layout, kv_len_dev, q_len_dev, n_batch, n_heads, head_dim, q_cap,
                                   softmax_scale, scratch, SR_NOALLOC_SCRATCH_BYTES, status_dev, stream);
+}
+
+extern "C" int sr_set_wait_limit_ns(uint64_t limit_ns) {
+    sr::g_wait_limit_ns.store(limit_ns ? limit_ns : sr::kWaitLimitNs, std::memory_order_relaxed);
+    return SR_OK;
+}
+
+extern "C" int sr_set_withheld_kv_tile(int32_t tile) {
+    if (tile < -1) return sr::set_error(SR_ERR_INVALID_ARG, "withheld tile must be >= -1");
+    sr::g_withheld_tile.store(tile, std::memory_order_relaxed);
+    return SR_OK;
 }

@@ -31,8 +31,15 @@ struct AttnLaunch {
     void *workspace;
     size_t workspace_bytes;
     cudaStream_t stream;
+    uint64_t wait_limit_ns;    // bound of every pipeline wait inside the kernels
+    int32_t withheld_tile;     // test hook: K tile whose load is withheld (-1: none)
 };
 int launch_chunk_attention(const AttnLaunch &a);
+
+// Library-wide settings of the attention launches (sr_set_wait_limit_ns,
+// sr_set_withheld_kv_tile): read at every launch.
+uint64_t attention_wait_limit_ns();
+int32_t attention_withheld_tile();
 
 // Work list of the attention kernel: units are (session, head, 256-row query
 // block); whole waves of units run one per CTA, and the units of a last
@@ -47,6 +54,14 @@ struct AttnSchedule {
 };
 AttnSchedule attention_schedule(int32_t n_batch, int32_t n_heads, int32_t head_dim, int32_t q_cap, int32_t sms);
 int attention_sm_count();
+// Units that run at once: CTA pairs at head_dim 128 (pair kernel), SMs at 64.
+int attention_slots(int32_t head_dim);
+int attention_pair_slots();
+int launch_pair_attention(const AttnLaunch &a, const AttnSchedule &sc);
+// Merge of the KV parts of split units (fp32 partials in the workspace).
+int launch_split_combine(const float *ws_o, const float *ws_ml, void *o, float *lse, const int32_t *q_len,
+                         int32_t n_full, int32_t split, int32_t tail_units, int32_t qb_per_head, int32_t n_heads,
+                         int32_t q_cap, int32_t head_dim, cudaStream_t stream);
 
 struct RopeLaunch {
     const void *x;
@@ -60,8 +75,11 @@ struct RopeLaunch {
     cudaStream_t stream;
     const float *gamma = nullptr;   // non-null: RMSNorm each head vector first
     float eps = 0.f;
-    void *y_raw = nullptr;          // optional normalised, unrotated copy
+    void *y_raw = nullptr;          // optional unrotated copy (normalised when gamma is set)
     int64_t rb = 0, rt = 0, rh = 0;
+    const double *t_origin = nullptr;   // optional device offset added to every t
+    const void *vx = nullptr;       // optional rows copied unrotated, strides of x -> y
+    void *vy = nullptr;
 };
 int launch_rope3d(const RopeLaunch &a);
 int rope_norm_max_heads(int head_dim);
@@ -79,6 +97,7 @@ struct GatherLaunch {
     sr_rope_cfg cfg;
     float out_scale;
     cudaStream_t stream;
+    const double *t_origin = nullptr;   // RoPE gather: optional offset added to every t
 };
 int launch_gather(const GatherLaunch &l);
 
@@ -93,6 +112,12 @@ struct PoolLaunch {
     int64_t pos_b;
     int32_t *slot_of_src;
     cudaStream_t stream;
+    void *k_rot = nullptr;          // optional fused RoPE output of the pooled K
+    const float *rot_pos = nullptr;
+    int64_t rot_pos_b = 0;
+    const double *t_origin = nullptr;
+    sr_rope_cfg rot_cfg{};
+    float rot_scale = 1.f;
 };
 int launch_history_compress(const PoolLaunch &a);
 
@@ -106,7 +131,14 @@ struct AppendLaunch {
     const int32_t *n_valid;
     int64_t sb, st, sh, psb;
     cudaStream_t stream;
+    void *k_rot = nullptr;          // optional: K rotated into this buffer (layout of k_buf)
+    const float *rot_pos = nullptr;
+    int64_t rot_pos_b = 0;
+    const double *t_origin = nullptr;
+    sr_rope_cfg rot_cfg{};
+    float rot_scale = 1.f;
 };
 int launch_kv_append(const AppendLaunch &a);
+int launch_clock_advance(double *clock, double frames, cudaStream_t stream);
 
 }  // namespace sr

@@ -54,16 +54,23 @@ struct RopeArgs {
     int64_t xb, xt, xh, yb, yt, yh, pb;
     // QK normalisation (norm kernels only): per-head RMSNorm with gain
     // gamma[D]; y_raw (optional) receives the normalised vector before RoPE
+    // (without normalisation: the input itself, a plain copy)
     const float *__restrict__ gamma;
     float eps;
     __nv_bfloat16 *__restrict__ y_raw;
     int64_t rb, rt, rh;
+    // optional fp64 offset added to every token's t (the stream clock)
+    const double *__restrict__ t_origin;
+    // optional second tensor copied unrotated with the strides of x -> y (V
+    // rows that travel with their K rows)
+    const __nv_bfloat16 *__restrict__ vx;
+    __nv_bfloat16 *__restrict__ vy;
 };
 
 // (cos, sin) * scale of one pair: the angle p * theta is formed in double and
 // reduced to [-pi, pi] in double, so its error does not grow with the
 // position's magnitude; the small remainder goes through fp32 sincosf.
-__device__ __forceinline__ float2 pair_rotation(const RopeTable &tab, int pair, float pt, float ph, float pw,
+__device__ __forceinline__ float2 pair_rotation(const RopeTable &tab, int pair, double pt, float ph, float pw,
                                                 float scale) {
     constexpr double kTwoPi = 6.283185307179586476925286766559;
     constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
@@ -77,7 +84,7 @@ __device__ __forceinline__ float2 pair_rotation(const RopeTable &tab, int pair, 
 
 // The token's four (cos, sin) pairs of chunk c (pairs 4c .. 4c+3), computed
 // as pair_rotation does; s_theta: the per-pair theta in shared memory.
-__device__ __forceinline__ void token_rotation(const double *s_theta, const RopeTable &tab, int c, float pt,
+__device__ __forceinline__ void token_rotation(const double *s_theta, const RopeTable &tab, int c, double pt,
                                                float ph, float pw, float scale, float (&cs)[4], float (&sn)[4]) {
     constexpr double kTwoPi = 6.283185307179586476925286766559;
     constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
@@ -153,15 +160,17 @@ __global__ void __launch_bounds__(128, kPasses <= 5 ? 8 : 4) rope3d_kernel(const
     __shared__ __align__(16) float2 s_rot[D / 2];
     __shared__ __align__(16) float s_gamma[kNorm ? D : 1];   // gains, read per pass (keeps registers free)
     if (threadIdx.x < D / 2) {
-        float pt = 0.f, ph = 0.f, pw = 0.f;
+        double pt = a.t_origin ? *a.t_origin : 0.0;
+        float ph = 0.f, pw = 0.f;
         if (a.pos) {
             const float *pp = a.pos + b * a.pb + 3 * static_cast<int64_t>(n);
-            pt = pp[0];
+            pt += static_cast<double>(pp[0]);
             ph = pp[1];
             pw = pp[2];
         }
         s_rot[threadIdx.x] = pair_rotation(tab, threadIdx.x, pt, ph, pw, a.out_scale);
     }
+
     if constexpr (kNorm) {
         if (threadIdx.x < D) s_gamma[threadIdx.x] = a.gamma[threadIdx.x];
     }
@@ -206,6 +215,9 @@ __global__ void __launch_bounds__(128, kPasses <= 5 ? 8 : 4) rope3d_kernel(const
             if (a.y_raw)
                 *reinterpret_cast<uint4 *>(a.y_raw + b * a.rb + n * a.rt + h * a.rh + c * 8) = pack8(f);
         }
+        if constexpr (!kNorm) {
+            if (a.y_raw) *reinterpret_cast<uint4 *>(a.y_raw + b * a.rb + n * a.rt + h * a.rh + c * 8) = u[i];
+        }
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             r[2 * k] = f[2 * k] * cs[k] - f[2 * k + 1] * sn[k];
@@ -214,9 +226,30 @@ __global__ void __launch_bounds__(128, kPasses <= 5 ? 8 : 4) rope3d_kernel(const
         *reinterpret_cast<uint4 *>(yt + h * a.yh) = pack8(r);
     }
     if constexpr (!kNorm) {   // with normalisation the host guarantees n_heads fits the passes above
+        for (int h = hp + kPasses * kHeadsPerPass; h < a.n_heads; h += kHeadsPerPass) {   // very many heads
+            const uint4 x8 = __ldg(reinterpret_cast<const uint4 *>(xt + h * a.xh));
+            if (a.y_raw) *reinterpret_cast<uint4 *>(a.y_raw + b * a.rb + n * a.rt + h * a.rh + c * 8) = x8;
+            *reinterpret_cast<uint4 *>(yt + h * a.yh) = rotate8(x8, cs, sn);
+        }
+    }
+    if (!kNorm && a.vx) {
+        // rows that travel unrotated with their K rows (V into the window):
+        // after the K rows, in the registers they used
+        const __nv_bfloat16 *vt = a.vx + b * a.xb + n * a.xt + c * 8;
+        __nv_bfloat16 *vo = a.vy + b * a.yb + n * a.yt + c * 8;
+        uint4 w[kPasses];
+#pragma unroll
+        for (int i = 0; i < kPasses; ++i) {
+            const int h = hp + i * kHeadsPerPass;
+            w[i] = h < a.n_heads ? __ldg(reinterpret_cast<const uint4 *>(vt + h * a.xh)) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int i = 0; i < kPasses; ++i) {
+            const int h = hp + i * kHeadsPerPass;
+            if (h < a.n_heads) *reinterpret_cast<uint4 *>(vo + h * a.yh) = w[i];
+        }
         for (int h = hp + kPasses * kHeadsPerPass; h < a.n_heads; h += kHeadsPerPass)   // very many heads
-            *reinterpret_cast<uint4 *>(yt + h * a.yh) =
-                rotate8(__ldg(reinterpret_cast<const uint4 *>(xt + h * a.xh)), cs, sn);
+            *reinterpret_cast<uint4 *>(vo + h * a.yh) = __ldg(reinterpret_cast<const uint4 *>(vt + h * a.xh));
     }
 }
 
@@ -232,6 +265,13 @@ struct PoolArgs {
     float *__restrict__ pos_out;
     int64_t pos_b;
     int64_t total;   // threads doing work per (batch, frame)
+    // optional fused RoPE of the pooled K (as rounded to bf16) into k_rot
+    // (strides of k_out) at rot_pos (layout of pos_out) + t_origin on t
+    __nv_bfloat16 *__restrict__ k_rot;
+    const float *__restrict__ rot_pos;
+    int64_t rot_pos_b;
+    const double *__restrict__ t_origin;
+    float rot_scale;
 };
 
 // One thread per (batch, frame, cell, head, 16-byte chunk); chunk fastest so a
@@ -240,7 +280,7 @@ struct PoolArgs {
 // flight together (members outside the grid are skipped); PH = PW = 0 reads
 // the window from the arguments.
 template <int D, int PH, int PW>
-__global__ void __launch_bounds__(256) pool_kernel(const PoolArgs a) {
+__global__ void __launch_bounds__(256) pool_kernel(const PoolArgs a, const RopeTable tab) {
     constexpr int kChunks = D / 8;
     const uint32_t idx = blockIdx.x * blockDim.x + threadIdx.x;   // (cell, head, chunk) of one frame
     if (idx >= static_cast<uint32_t>(a.total)) return;
@@ -294,7 +334,21 @@ __global__ void __launch_bounds__(256) pool_kernel(const PoolArgs a) {
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = acc[e] / count;
-        *reinterpret_cast<uint4 *>(dst + out_off) = pack8(acc);
+        const uint4 pooled = pack8(acc);
+        *reinterpret_cast<uint4 *>(dst + out_off) = pooled;
+        if (which == 0 && a.k_rot) {
+            // the pooled key enters its slot rotated once, from its bf16 value
+            const float *pp = a.rot_pos + b * a.rot_pos_b + 3 * (static_cast<int64_t>(f) * a.cells + j);
+            const double pt = (a.t_origin ? *a.t_origin : 0.0) + static_cast<double>(pp[0]);
+            float cs[4], sn[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float2 r = pair_rotation(tab, c * 4 + k, pt, pp[1], pp[2], a.rot_scale);
+                cs[k] = r.x;
+                sn[k] = r.y;
+            }
+            *reinterpret_cast<uint4 *>(a.k_rot + out_off) = rotate8(pooled, cs, sn);
+        }
     }
     if (a.pos_out && h == 0 && c == 0) {
         float *pp = a.pos_out + b * a.pos_b + 3 * (static_cast<int64_t>(f) * a.cells + j);
@@ -372,6 +426,7 @@ struct GatherArgs {
     int64_t src_t, src_h, dst_b, dst_s, dst_h, pos_b;
     int64_t total;                     // threads per batch entry: slots x D/8
     float out_scale;                   // RoPE gather only
+    const double *__restrict__ t_origin;   // RoPE gather only: optional offset added to every t
 };
 
 constexpr int kGatherHeads = 8;   // head rows a thread keeps in flight
@@ -410,7 +465,8 @@ __global__ void __launch_bounds__(256) gather_kernel(const GatherArgs a, const R
     float cs[4], sn[4];
     if constexpr (kRope) {
         const float *pp = a.src_pos + 3 * static_cast<int64_t>(t);
-        token_rotation(s_theta, tab, c, pp[0], pp[1], pp[2], a.out_scale, cs, sn);
+        const double pt = (a.t_origin ? *a.t_origin : 0.0) + static_cast<double>(pp[0]);
+        token_rotation(s_theta, tab, c, pt, pp[1], pp[2], a.out_scale, cs, sn);
     }
     for (int h0 = 0; h0 < a.n_heads; h0 += kGatherHeads) {
         uint4 u[kGatherHeads];
@@ -460,7 +516,7 @@ template <int D>
 int gather_launch(const GatherLaunch &l) {
     GatherArgs a{l.dst, l.src, l.idx, l.src_pos, l.dst_pos, l.n_slots, l.n_heads,
                  l.src_t, l.src_h, l.dst_b, l.dst_s, l.dst_h, l.pos_b,
-                 static_cast<int64_t>(l.n_slots) * (D / 8), l.out_scale};
+                 static_cast<int64_t>(l.n_slots) * (D / 8), l.out_scale, l.t_origin};
     if (a.total > 0x7fffffff || l.n_batch > 65535)
         return set_error(SR_ERR_INVALID_ARG, "gather/scatter: too many slots or batch entries");
     const dim3 grid(static_cast<unsigned>((a.total + 255) / 256), l.n_batch);
@@ -480,7 +536,8 @@ int rope_launch(const RopeLaunch &l) {
     const RopeTable tab = make_rope_table(l.cfg);
     RopeArgs a{static_cast<const __nv_bfloat16 *>(l.x), static_cast<__nv_bfloat16 *>(l.y), l.pos, l.n_valid,
                l.n_heads, l.out_scale, l.xb, l.xt, l.xh, l.yb, l.yt, l.yh, l.pb,
-               l.gamma, l.eps, static_cast<__nv_bfloat16 *>(l.y_raw), l.rb, l.rt, l.rh};
+               l.gamma, l.eps, static_cast<__nv_bfloat16 *>(l.y_raw), l.rb, l.rt, l.rh,
+               l.t_origin, static_cast<const __nv_bfloat16 *>(l.vx), static_cast<__nv_bfloat16 *>(l.vy)};
     dim3 grid(l.n_tokens, l.n_batch);
     // passes of 128 / (D/8) heads each: instantiated for 1..8 (more heads run
     // the extra passes in a loop, without normalisation only)
@@ -519,17 +576,23 @@ int pool_launch(const PoolLaunch &l) {
     a.frame_t = l.frame_t;
     a.pos_out = l.pos_out;
     a.pos_b = l.pos_b;
+    a.k_rot = static_cast<__nv_bfloat16 *>(l.k_rot);
+    a.rot_pos = l.rot_pos;
+    a.rot_pos_b = l.rot_pos_b;
+    a.t_origin = l.t_origin;
+    a.rot_scale = l.rot_scale;
     a.total = static_cast<int64_t>(a.cells) * l.n_heads * (D / 8);   // threads per frame
     if (a.total > 0x7fffffff || l.n_frames > 65535 || l.n_batch > 65535)
         return set_error(SR_ERR_INVALID_ARG, "history_compress: too many cells, frames or sessions");
     if (a.total > 0) {
         const dim3 blocks(static_cast<unsigned>((a.total + 255) / 256), l.n_frames, l.n_batch);
+        const RopeTable tab = l.k_rot ? make_rope_table(l.rot_cfg) : RopeTable{};
         if (a.pool_h == 2 && a.pool_w == 2)
-            pool_kernel<D, 2, 2><<<blocks, 256, 0, l.stream>>>(a);
+            pool_kernel<D, 2, 2><<<blocks, 256, 0, l.stream>>>(a, tab);
         else if (a.pool_h == 4 && a.pool_w == 4)
-            pool_kernel<D, 4, 4><<<blocks, 256, 0, l.stream>>>(a);
+            pool_kernel<D, 4, 4><<<blocks, 256, 0, l.stream>>>(a, tab);
         else
-            pool_kernel<D, 0, 0><<<blocks, 256, 0, l.stream>>>(a);
+            pool_kernel<D, 0, 0><<<blocks, 256, 0, l.stream>>>(a, tab);
     }
     if (l.slot_of_src) {
         const int64_t n = static_cast<int64_t>(l.n_frames) * l.cfg.grid_h * l.cfg.grid_w;
@@ -544,6 +607,31 @@ int pool_launch(const PoolLaunch &l) {
 
 template <int D>
 int append_launch(const AppendLaunch &l) {
+    if (l.k_rot) {
+        // K rotated into k_rot (and copied raw into k_buf if given), V copied:
+        // the RoPE kernel, one CTA per token, head-major destination rows
+        const int64_t hb = static_cast<int64_t>(l.buf_tokens) * D;   // head stride of the buffers
+        const int64_t bb = static_cast<int64_t>(l.n_heads) * hb;      // batch stride
+        const int64_t off = static_cast<int64_t>(l.dst_token) * D;
+        RopeLaunch r{l.k_src, static_cast<__nv_bfloat16 *>(l.k_rot) + off, l.rot_pos, l.n_valid, l.n_batch,
+                     l.n_tokens, l.n_heads, D, l.rot_cfg, l.rot_scale, l.sb, l.st, l.sh, bb, D, hb,
+                     l.rot_pos_b, l.stream};
+        r.y_raw = l.k_buf && l.k_src ? static_cast<__nv_bfloat16 *>(l.k_buf) + off : nullptr;
+        r.rb = bb;
+        r.rt = D;
+        r.rh = hb;
+        r.t_origin = l.t_origin;
+        if (l.v_src) {
+            r.vx = l.v_src;
+            r.vy = static_cast<__nv_bfloat16 *>(l.v_buf) + off;
+        }
+        int rc = rope_launch<D, false>(r);
+        if (rc != SR_OK || !l.pos_src) return rc;
+        AppendLaunch pl = l;   // positions only, by the plain copy
+        pl.k_src = pl.v_src = nullptr;
+        pl.k_rot = nullptr;
+        return append_launch<D>(pl);
+    }
     AppendArgs a{};
     a.k_buf = static_cast<__nv_bfloat16 *>(l.k_buf);
     a.v_buf = static_cast<__nv_bfloat16 *>(l.v_buf);
@@ -566,7 +654,15 @@ int append_launch(const AppendLaunch &l) {
     return e == cudaSuccess ? SR_OK : set_cuda_error("kv_append launch", e);
 }
 
+__global__ void clock_advance_kernel(double *clock, double frames) { *clock += frames; }
+
 }  // namespace
+
+int launch_clock_advance(double *clock, double frames, cudaStream_t stream) {
+    clock_advance_kernel<<<1, 1, 0, stream>>>(clock, frames);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SR_OK : set_cuda_error("stream_clock_advance launch", e);
+}
 
 int launch_rope3d(const RopeLaunch &l) {
     if (l.gamma) return l.head_dim == 128 ? rope_launch<128, true>(l) : rope_launch<64, true>(l);

@@ -28,9 +28,14 @@ Per step, on every rank:
           the send buffer [world*S, Hn, D]
   a2a     back: recv_o[j] = O of head group j for this rank's tokens
   unpack  recv_o [world, S, Hn, D] -> out [S, H, D]
-The pack and unpack are layout copies; the exchanges are NCCL all-to-alls
-over NVLink (``torch.distributed.all_to_all_single``).  The phases are
-separate methods so that a test can run several ranks in one process.
+The pack and unpack are layout copies done by the library's index gather
+and scatter (sr_gather_tokens: one launch per tensor; sr_scatter_tokens: one
+launch), with a fixed index table: slot (j, t) of the send buffer is token t
+of head group j, i.e. row t * world + j of the rank's [n, H, D] tokens viewed
+as [n * world, Hn, D].  The exchanges are NCCL all-to-alls over NVLink
+(``torch.distributed.all_to_all_single``).  The phases are separate methods
+so that a test can run several ranks in one process; ranks on the CPU (the
+multi-process tests over gloo) re-lay out with torch copies instead.
 """
 from __future__ import annotations
 
@@ -104,6 +109,13 @@ class UlyssesAttention:
         self.recv = torch.zeros(N, S, 3, Hn, D, **kw)
         self.o_send = torch.zeros(N * S, Hn, D, **kw)
         self.o_recv = torch.zeros(N, S, Hn, D, **kw)
+        # slot (head group j, token t) <-> row t * world + j of the tokens viewed
+        # [n * world, Hn, D]; slots past this rank's n tokens: -1 (zero / skipped)
+        lo, hi = self.plan.tokens_of(rank)
+        t = torch.arange(S, dtype=torch.int64)
+        idx = t[None, :] * N + torch.arange(N, dtype=torch.int64)[:, None]
+        idx[:, hi - lo:] = -1
+        self.idx = idx.to(torch.int32).contiguous().to(self.device)
 
     # ------------------------------------------------------------ phases
     def load_window(self, inp) -> None:
@@ -117,8 +129,13 @@ class UlyssesAttention:
         lo, hi = self.plan.tokens_of(self.rank)
         if n != hi - lo:
             raise ValueError(f"rank {self.rank} holds {hi - lo} tokens, got {n}")
-        for c, x in enumerate((q, k, v)):
-            self.send[:, :n, c].copy_(x.view(n, self.world, self.Hn, self.D).transpose(0, 1))
+        if self.device.type == "cuda":
+            from . import capi
+            for c, x in enumerate((q, k, v)):
+                capi.sr_gather_tokens(self.send[:, :, c], x.reshape(n * self.world, self.Hn, self.D), self.idx)
+        else:   # CPU ranks of the multi-process tests
+            for c, x in enumerate((q, k, v)):
+                self.send[:, :n, c].copy_(x.view(n, self.world, self.Hn, self.D).transpose(0, 1))
         return self.send
 
     def attend(self, marks=None) -> torch.Tensor:
@@ -140,7 +157,11 @@ class UlyssesAttention:
         n = hi - lo
         if out is None:
             out = torch.empty(n, self.H, self.D, dtype=torch.bfloat16, device=self.device)
-        out.view(n, self.world, self.Hn, self.D).copy_(self.o_recv[:, :n].transpose(0, 1))
+        if self.device.type == "cuda":
+            from . import capi
+            capi.sr_scatter_tokens(out.view(n * self.world, self.Hn, self.D), self.o_recv, self.idx)
+        else:   # CPU ranks of the multi-process tests
+            out.view(n, self.world, self.Hn, self.D).copy_(self.o_recv[:, :n].transpose(0, 1))
         return out
 
     # ------------------------------------------------------------ the step

@@ -100,12 +100,15 @@ class RingWindowAttention:
             self.kv_len_phase.append(torch.from_numpy(lens).to(self.device))
         ws = capi.sr_chunk_attention_workspace_bytes(W, H, D, self.q_cap)
         self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, **kw) if ws else None
-        # positions of the current frames: (f, row, col) + t0 on the t axis,
-        # formed on the device so that a call never waits for the host
+        # positions of the current frames: the fixed table (f, row, col) plus
+        # the call's first frame index t0 on the t axis, which the rotating
+        # kernels add themselves from a device clock (fp64): a call never waits
+        # for the host and a replayed graph sees the new t0.  The clock is
+        # advanced by frames_per_call at the start of every call's prepare, so
+        # consecutive calls need no host write; a jump in t0 sets it directly.
         self.pos_base = self.frame_positions(0)
-        self.t_axis = torch.tensor([1.0, 0.0, 0.0], **kw)
-        self.t0_dev = torch.zeros(1, **kw)
-        self.pos_cur = torch.zeros_like(self.pos_base)
+        self.t0_dev = torch.zeros(1, dtype=torch.float64, **kw)
+        self.t0_next = None   # t0 the device clock reaches at the next advance
         self.calls = 0
         self.graphs = {}
 
@@ -125,16 +128,24 @@ class RingWindowAttention:
         rotated on the way into its ring slot) and the partition of the
         queries (rotated on the way): one gather launch each."""
         S = self.slot_cap
-        torch.addcmul(self.pos_base, self.t_axis, self.t0_dev, out=self.pos_cur)
+        capi.sr_stream_clock_advance(self.t0_dev, float(self.fpc), stream=stream)
         for f in range(self.fpc):
             sl = (slot0 + f) % self.slots
             ring_k = self.k_ring[:, :, sl * S:(sl + 1) * S].permute(0, 2, 1, 3)
             ring_v = self.v_ring[:, :, sl * S:(sl + 1) * S].permute(0, 2, 1, 3)
             capi.sr_gather_tokens(ring_v, v, self.idx_kv[f], stream=stream)
-            capi.sr_gather_rope3d_tokens(ring_k, k, self.idx_kv[f], self.pos_cur, self.split, self.base,
-                                         stream=stream)
-        capi.sr_gather_rope3d_tokens(self.q_att.permute(0, 2, 1, 3), q, self.idx_q, self.pos_cur, self.split,
-                                     self.base, stream=stream)
+            capi.sr_gather_rope3d_tokens(ring_k, k, self.idx_kv[f], self.pos_base, self.split, self.base,
+                                         t_origin=self.t0_dev, stream=stream)
+        capi.sr_gather_rope3d_tokens(self.q_att.permute(0, 2, 1, 3), q, self.idx_q, self.pos_base, self.split,
+                                     self.base, t_origin=self.t0_dev, stream=stream)
+
+    def _set_t0(self, t0: int) -> None:
+        """Make the next advance of the device clock land on t0: nothing to do
+        for consecutive calls; otherwise one host-to-device copy (in stream
+        order, no kernel)."""
+        if self.t0_next != t0:
+            self.t0_dev.copy_(torch.tensor([float(t0 - self.fpc)], dtype=torch.float64))
+        self.t0_next = t0 + self.fpc
 
     def _attend(self, phase: int, stream=None) -> None:
         S = self.slot_cap
@@ -156,7 +167,7 @@ class RingWindowAttention:
         if out is None:
             out = torch.zeros_like(q)
         slot0, phase = self._state()
-        self.t0_dev.fill_(float(t0))
+        self._set_t0(t0)
         self._prepare(q, k, v, slot0, stream)
         _mark(marks, 0, stream)
         self._attend(phase, stream)
@@ -190,7 +201,7 @@ class RingWindowAttention:
             self.graphs[key] = gs
             return out
         gs = self.graphs[key]
-        self.t0_dev.fill_(float(t0))
+        self._set_t0(t0)
         gs[0].replay()
         _mark(marks, 0, None)
         gs[1].replay()

@@ -21,9 +21,16 @@ Sources:
 Readings (the pages leave them open): window-relative positions with the
 chunk's frames at t = 0, 1, ... and the context frames at t = -n .. -1 (the
 sink earliest); audio token i at t = i * 6 / 40, h = w = 0; pooled cells at
-(t, mean member row, mean member col); the prompt unrotated; K is kept
-pre-RoPE in the window (``k_raw``) and rotated into ``k_att`` with the current
-template, so re-positioning never compounds rounding.  After a chunk its
+(t, mean member row, mean member col); the prompt at position 0.  q . k after
+RoPE depends on position differences only, so every rotation adds a stream
+clock (fp64, on the device) to the template t: a slide of n frames advances
+the clock by n while the frames' template t fall by n, so a history frame
+keeps its rotated keys, rotated once when it enters a ring slot (pooled or
+appended, fused into that call).  Only what floats with the chunk is rotated
+every step: the chunk's keys (fused into their append), the queries and the
+prefix (prompt and sink, whose template places stay fixed relative to the
+chunk).  K is also kept pre-RoPE (``k_raw``) where it is pooled later, so
+rotation never compounds rounding.  After a chunk its
 clean frames become the newest history and every tier hands its oldest
 frames to the next older tier (re-pooled), the oldest tier dropping its
 oldest: each of tier0.., recent is a ring of frame slots, so only the frames
@@ -169,6 +176,9 @@ class StreamingWindow:
         self.o = torch.zeros(B, self.q_cap, H, D, dtype=torch.bfloat16, **kw)
         self.lse = torch.zeros(B, H, self.q_cap, dtype=torch.float32, **kw)
         self.status = torch.zeros(1, dtype=torch.int32, **kw)
+        # stream clock: t of the current chunk's first latent frame on the
+        # time axis every rotation shares (template t + clock)
+        self.clock = torch.zeros(1, dtype=torch.float64, **kw)
         ws = capi.sr_chunk_attention_workspace_bytes(B, H, D, self.q_cap) if self.device.type == "cuda" else 0
         self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, **kw) if ws else None
         lens = np.array([[p.lengths[s] for s in self.segments] for p in self.plans], dtype=np.int32)
@@ -246,40 +256,67 @@ class StreamingWindow:
                                       pos, stream=stream)
                     fill[role] += ntok
                     f += 1
-        # the prompt is never re-positioned: rotate (identity) once
-        self._rope(self.seg_view(self.k_raw, "prompt"), self.seg_view(self.k_att, "prompt"), None, key=True,
-                   n_valid=self.seg_valid[0], stream=stream)
         # chunk positions are the fixed template
         off = self.seg["chunk"][0]
         self.pos[:, off:off + self.q_cap].copy_(self.q_pos)
+        # a reload restarts the stream clock; every key of the loaded window is
+        # rotated once (padded slots hold zeros and stay zeros)
+        self.clock.zero_()
+        self._rope(self.k_raw.permute(0, 2, 1, 3), self.k_att.permute(0, 2, 1, 3), self.pos, key=True,
+                   stream=stream)
 
     # ---------------------------------------------------------------- the step
-    def append_chunk(self, k: torch.Tensor, v: torch.Tensor, stream=None) -> None:
-        """a2: chunk K (pre-RoPE) and V [B, q_cap, H, D] into the chunk segment."""
-        capi.sr_kv_append(self.k_raw, self.v, None, self.seg["chunk"][0], k, v, None, n_valid=self.q_len,
-                          stream=stream)
+    def append_chunk(self, k: torch.Tensor, v: torch.Tensor, stream=None, rotate: bool = None) -> None:
+        """a2 (with a3 of the chunk keys): chunk K and V [B, q_cap, H, D] into
+        the chunk segment.  By default the keys are rotated on the way in
+        (k_att; the chunk's pre-RoPE keys are never pooled, so k_raw is not
+        written); with rotate=False, or with QK normalisation, K goes to
+        k_raw unrotated for a later whole-window rotation."""
+        if rotate is None:
+            rotate = self.qk_norm is None
+        off = self.seg["chunk"][0]
+        if rotate:
+            rot = capi.RopeOut(self.k_att, self.q_pos, self.split, self.base, t_origin=self.clock)
+            capi.sr_kv_append(None, self.v, None, off, k, v, None, n_valid=self.q_len, rot=rot, stream=stream)
+        else:
+            capi.sr_kv_append(self.k_raw, self.v, None, off, k, v, None, n_valid=self.q_len, stream=stream)
 
     def rotate(self, q: torch.Tensor, stream=None) -> None:
-        """a3: RoPE of the chunk queries into q_att, and of every non-prompt
-        window slot from k_raw into k_att with the current template.  The
-        window part is one launch over the contiguous slots after the prompt;
-        padded slots hold zeros (position 0) and stay zeros."""
+        """a3: RoPE of the chunk queries into q_att, and of the keys whose
+        template places float with the chunk: the prefix (prompt, sink), one
+        launch over its contiguous slots.  With QK normalisation every window
+        key is normalised and rotated again instead (from k_raw)."""
         self._rope(q, self.q_att.permute(0, 2, 1, 3), self.q_pos, key=False, n_valid=self.q_len, stream=stream)
-        self.rotate_keys(stream)
+        if self.qk_norm is None:
+            self.rotate_prefix(stream)
+        else:
+            self.rotate_keys(stream)
+
+    def prefix_slots(self) -> int:
+        """Slots of the prefix segments (prompt, then sink) at the buffer start."""
+        return sum(c for name, c in zip(self.segments, self.caps) if name in ("prompt", "sink"))
+
+    def rotate_prefix(self, stream=None) -> None:
+        """RoPE of the prefix slots (prompt, sink) from k_raw into k_att at the
+        current clock (one launch)."""
+        n = self.prefix_slots()
+        self._rope(self.k_raw[:, :, :n].permute(0, 2, 1, 3), self.k_att[:, :, :n].permute(0, 2, 1, 3),
+                   self.pos[:, :n], key=True, stream=stream)
 
     def rotate_keys(self, stream=None) -> None:
-        """RoPE of every non-prompt window slot from k_raw into k_att (one launch)."""
-        off = self.seg["prompt"][1]
-        self._rope(self.k_raw[:, :, off:].permute(0, 2, 1, 3), self.k_att[:, :, off:].permute(0, 2, 1, 3),
-                   self.pos[:, off:], key=True, stream=stream)
+        """RoPE of every window slot from k_raw into k_att at the current clock
+        (one launch)."""
+        self._rope(self.k_raw.permute(0, 2, 1, 3), self.k_att.permute(0, 2, 1, 3), self.pos, key=True,
+                   stream=stream)
 
     def _rope(self, x, y, pos, key: bool, n_valid=None, stream=None) -> None:
         if self.qk_norm is None:
-            capi.sr_rope3d_apply(x, y, pos, self.split, self.base, n_valid=n_valid, stream=stream)
+            capi.sr_rope3d_apply(x, y, pos, self.split, self.base, n_valid=n_valid, t_origin=self.clock,
+                                 stream=stream)
         else:
             gq, gk, eps = self.qk_norm
             capi.sr_qknorm_rope3d_apply(x, y, gk if key else gq, eps, pos, self.split, self.base, n_valid=n_valid,
-                                        stream=stream)
+                                        t_origin=self.clock, stream=stream)
 
     def attend(self, stream=None, out: torch.Tensor = None, marks=None) -> torch.Tensor:
         """a4: fused chunk attention -> o [B, q_cap, H, D] (and lse); `out`
@@ -363,7 +400,7 @@ class StreamingWindow:
         pos, lens, kv_len = self._prefix_meta
         assert n_pre == pos.shape[1], "q_prefix must cover prompt + sink tokens"
         q_att, o, lse, ws = self._scratch("prefix", n_pre)
-        self.rotate_keys(stream)
+        self.rotate_prefix(stream)
         self._rope(q_prefix, q_att.permute(0, 2, 1, 3), pos, key=False, n_valid=lens, stream=stream)
         capi.sr_chunk_attention_fwd(q_att, self.k_att, self.v, o, lse, self.caps, kv_len, lens, self.scale,
                                     self.status, workspace=ws, stream=stream)
@@ -397,7 +434,7 @@ class StreamingWindow:
             rows = slice(j * ft, min((j + m) * ft, n_rec))
             capi.sr_kv_append(self.k_raw, self.v, None, off_r + slot * ft, k_recent[:, rows], v_recent[:, rows],
                               None, stream=stream)
-        self.append_chunk(k, v, stream)
+        self.append_chunk(k, v, stream, rotate=False)
         n_mov = n_rec + self.q_cap
         q_att, o, lse, ws = self._scratch("moving", n_mov)
         # chunk queries straight into their rows of the moving query buffer
@@ -572,28 +609,116 @@ class StreamingWindow:
         elif n != self.slide_frames:
             raise ValueError(f"every slide must move {self.slide_frames} frames")
         ops, nxt = self.slide_ops(self.ring_ptr)
-        self._launch_slide(ops, k_clean, v_clean, stream)
         self.ring_ptr = nxt
-        self.pos = self._phases[tuple(nxt.values())]
+        self.pos = self._phases[tuple(nxt.values())]   # the new state's template: the entering keys' places
+        capi.sr_stream_clock_advance(self.clock, float(n), stream=stream)
+        self._launch_slide(ops, k_clean, v_clean, stream)
 
     def _launch_slide(self, ops, k_clean, v_clean, stream=None) -> None:
-        """The kernel calls of one slide plan (no host state changes)."""
+        """The kernel calls of one slide plan (no host state changes).  The
+        keys entering a ring slot are rotated on the way in at the template
+        of self.pos (the new ring state) plus the clock, except with QK
+        normalisation, whose every step re-rotates the whole window."""
         ft = self.plans[0].frame_tokens
+        rotate = self.qk_norm is None
         for op in ops:
             if op[0] == "pool":
                 _, src, fs, dst, fd, m, grid, pool = op
+                rot = None
+                if rotate:
+                    r = self.rings[dst]
+                    off = self.seg[dst][0] + fd * r["tok"]
+                    rot = capi.RopeOut(self._ring_frames(self.k_att, dst, fd, m), self.pos[:, off:off + m * r["tok"]],
+                                       self.split, self.base, t_origin=self.clock)
                 capi.sr_history_compress(self._ring_frames(self.k_raw, src, fs, m),
                                          self._ring_frames(self.v, src, fs, m),
                                          self._ring_frames(self.k_raw, dst, fd, m),
-                                         self._ring_frames(self.v, dst, fd, m), grid, pool, stream=stream)
+                                         self._ring_frames(self.v, dst, fd, m), grid, pool, rot=rot, stream=stream)
             else:
                 _, fr, fc, m = op
-                capi.sr_kv_append(self.k_raw, self.v, None, self.seg["recent"][0] + fr * ft,
-                                  k_clean[:, fc * ft:(fc + m) * ft], v_clean[:, fc * ft:(fc + m) * ft], None,
-                                  stream=stream)
+                off = self.seg["recent"][0] + fr * ft
+                rot = capi.RopeOut(self.k_att, self.pos[:, off:off + m * ft], self.split, self.base,
+                                   t_origin=self.clock) if rotate else None
+                capi.sr_kv_append(self.k_raw, self.v, None, off, k_clean[:, fc * ft:(fc + m) * ft],
+                                  v_clean[:, fc * ft:(fc + m) * ft], None, rot=rot, stream=stream)
+
+    def step_ops(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, k_clean: torch.Tensor = None,
+                 v_clean: torch.Tensor = None, ptr=None):
+        """The library calls of one streaming step before the attention, in
+        launch order: (name, algorithmic bytes, branch, launch) with launch()
+        issuing the call on the current stream.  With k_clean / v_clean the
+        stream clock advance and the window slide from ring state ``ptr`` come
+        first (its pooling and append calls); then the chunk append, the RoPE
+        of the chunk queries and the RoPE of the prefix (or, with QK
+        normalisation, of the whole window).  Algorithmic bytes count each
+        valid token's data read or written once (positions included where a
+        call reads them), the measure of the HBM roofline of each call.
+        Branch 0 runs first; the calls of branches 1, 2, ... depend only on
+        branch 0 and on earlier calls of their own branch, so the branches may
+        run concurrently (a last branch 4, the whole-window RoPE, waits for
+        all the others)."""
+        H, D, B = self.H, self.D, self.B
+        row = H * D * 2                                   # bytes of one token's K (or V) row
+        fused = self.qk_norm is None                      # keys rotated on entry (else re-rotated every step)
+        out_rows = 3 if fused else 2                      # K before RoPE, K rotated, V
+        ops = []
+        if k_clean is not None:
+            ft = self.plans[0].frame_tokens
+            n = self.slide_frames
+            ops.append(("stream clock", None, 0, lambda: capi.sr_stream_clock_advance(self.clock, float(n))))
+            for op in self.slide_ops(ptr)[0]:
+                if op[0] == "pool":
+                    _, src, _, dst, _, m, _, _ = op
+                    t_src, t_dst = m * self.rings[src]["tok"], m * self.rings[dst]["tok"]
+                    nb = B * (2 * t_src * row + out_rows * t_dst * row + (12 * t_dst if fused else 0))
+                    ops.append((f"pool {src}->{dst}", nb, 1,
+                                lambda op=op: self._launch_slide([op], k_clean, v_clean)))
+                else:
+                    t = op[3] * ft
+                    nb = B * (2 * t * row + out_rows * t * row + (12 * t if fused else 0))
+                    ops.append(("append clean frames", nb, 1,
+                                lambda op=op: self._launch_slide([op], k_clean, v_clean)))
+        n_q = int(sum(p.chunk_len for p in self.plans))
+        ops.append(("append chunk" + (" + RoPE" if fused else ""), 2 * 2 * n_q * row + (12 * n_q if fused else 0),
+                    2, lambda: self.append_chunk(k, v)))
+        ops.append(("rope chunk queries", n_q * (2 * row + 12), 3,
+                    lambda: self._rope(q, self.q_att.permute(0, 2, 1, 3), self.q_pos, key=False, n_valid=self.q_len)))
+        if fused:
+            n_pre = int(sum(p.lengths["prompt"] + p.lengths.get("sink", 0) for p in self.plans))
+            ops.append(("rope prefix keys", n_pre * (2 * row + 12), 3, lambda: self.rotate_prefix()))
+        else:   # every key is re-rotated from k_raw: after the slide and the chunk append
+            n_keys = int(self.lengths.sum())
+            ops.append(("rope window keys", n_keys * (2 * row + 12), 4, lambda: self.rotate_keys()))
+        return ops
+
+    def _launch_branches(self, ops) -> None:
+        """Issue step_ops entries: branch 0 on the current stream, every other
+        branch on a side stream forked from it (joined back at the end);
+        branch 4 (the whole-window RoPE) also waits for every other branch.
+        Captured into a CUDA graph, the branches become parallel paths the
+        device may run at the same time."""
+        cur = torch.cuda.current_stream()
+        for _, _, br, launch in ops:
+            if br == 0:
+                launch()
+        side = self.__dict__.setdefault("_side_streams", {})
+        ends = []
+        for b in sorted({br for _, _, br, _ in ops if br > 0}):
+            st = side.setdefault(b, torch.cuda.Stream(device=self.device))
+            st.wait_stream(cur)
+            if b == 4:
+                for e in ends:
+                    st.wait_stream(e)
+            with torch.cuda.stream(st):
+                for _, _, br, launch in ops:
+                    if br == b:
+                        launch()
+            ends.append(st)
+        for st in ends:
+            cur.wait_stream(st)
 
     def graph_step(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, k_clean: torch.Tensor = None,
-                   v_clean: torch.Tensor = None, marks=None) -> torch.Tensor:
+                   v_clean: torch.Tensor = None, marks=None, op_marks=None) -> torch.Tensor:
         """advance(k_clean, v_clean) (when given) and step(q, k, v), replayed
         from CUDA graphs: no per-launch host work, and the launches follow
         each other without gaps.
@@ -602,7 +727,13 @@ class StreamingWindow:
         state is captured the first time it occurs, after that call has run
         eagerly; later calls replay two graphs on the current stream (the
         slide, append and RoPE; the attention), with `marks` recorded around
-        the second.  Returns the window's output buffer."""
+        the second.  In the first graph the independent calls (see step_ops)
+        are parallel branches.  ``op_marks`` (a list the call fills) instead
+        replays every call of the step from a graph of its own, one after the
+        other, with a CUDA event recorded before each and after the attention:
+        it receives (name, algorithmic bytes, start event, end event) per call
+        and ("attention", None, start, end) last -- the per-call timing of the
+        step.  Returns the window's output buffer."""
         slide = k_clean is not None
         key = tuple(self.ring_ptr.values()) if slide and hasattr(self, "rings") else None
         graphs = self.__dict__.setdefault("_step_graphs", {})
@@ -613,26 +744,41 @@ class StreamingWindow:
             torch.cuda.synchronize()
             if slide and key is None:    # the rings were set up by this first slide: capture from the next one
                 return self.o
-            ops = self.slide_ops(dict(zip(self.rings, key)))[0] if slide else []
+            ops = self.step_ops(q, k, v, k_clean, v_clean, dict(zip(self.rings, key)) if slide else None)
             g_prep, g_attn = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
             with torch.cuda.graph(g_prep):   # self.pos already holds the next state's table
-                if slide:
-                    self._launch_slide(ops, k_clean, v_clean)
-                self.append_chunk(k, v)
-                self.rotate(q)
+                self._launch_branches(ops)
             with torch.cuda.graph(g_attn):
                 self.attend()
-            graphs[key] = (g_prep, g_attn)
+            per_op = []
+            for name, nbytes, _, launch in ops:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    launch()
+                per_op.append((name, nbytes, g))
+            graphs[key] = (g_prep, g_attn, per_op)
             return self.o
-        g_prep, g_attn = graphs[key]
+        g_prep, g_attn, per_op = graphs[key]
         if slide:
             nxt = self.slide_ops(self.ring_ptr)[1]
             self.ring_ptr = nxt
             self.pos = self._phases[tuple(nxt.values())]
-        g_prep.replay()
-        _mark(marks, 0, None)
+        if op_marks is None:
+            g_prep.replay()
+            _mark(marks, 0, None)
+            g_attn.replay()
+            _mark(marks, 1, None)
+            return self.o
+        stream = torch.cuda.current_stream()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(per_op) + 2)]
+        for i, (_, _, g) in enumerate(per_op):
+            evs[i].record(stream)
+            g.replay()
+        evs[-2].record(stream)
         g_attn.replay()
-        _mark(marks, 1, None)
+        evs[-1].record(stream)
+        op_marks.extend((name, nbytes, evs[i], evs[i + 1]) for i, (name, nbytes, _) in enumerate(per_op))
+        op_marks.append(("attention", None, evs[-2], evs[-1]))
         return self.o
 
     def recent_slot_order(self) -> List[int]:
@@ -641,6 +787,56 @@ class StreamingWindow:
             return list(range(_ceil_div(self.plans[0].lengths.get("recent", 0), self.plans[0].frame_tokens)))
         r = self.rings["recent"]
         return [(self.ring_ptr["recent"] + j) % r["frames"] for j in range(r["frames"])]
+
+    # ---------------------------------------------------------------- checkpoint / resume
+    # "StreamRender-H3" (molayo1419.me), inference acceleration section: the
+    # per-layer KV buffers are persistent and updated in place, so a session's
+    # whole state is those buffers plus the host-side ring pointers and the
+    # position table they select.
+    def export_state(self) -> dict:
+        """Snapshot of the session state on the host (synchronises with the
+        device): the window buffers (keys before and after RoPE, values), the
+        stream clock, the position table in use and, once the window has slid,
+        the ring pointers,
+        the frames per slide and the position table of the loaded window that
+        every ring state's table is built from.  ``import_state`` on a window
+        made from the same specs continues the stream bit for bit."""
+        torch.cuda.synchronize(self.device)
+        st = {"shape": (self.B, self.H, self.cap_total, self.D), "segments": list(self.segments),
+              "caps": list(self.caps), "lengths": self.lengths.copy(),
+              "k_raw": self.k_raw.cpu(), "k_att": self.k_att.cpu(), "v": self.v.cpu(), "pos": self.pos.cpu(),
+              "clock": self.clock.cpu()}
+        if hasattr(self, "rings"):
+            st.update(ring_ptr=dict(self.ring_ptr), slide_frames=int(self.slide_frames),
+                      pos_loaded=self._pos_loaded.cpu())
+        return st
+
+    def import_state(self, st: dict) -> None:
+        """Restore a snapshot taken by ``export_state`` (same specs: shapes,
+        segments and valid lengths must agree).  Captured step graphs are
+        dropped; the next slide continues from the saved ring pointers."""
+        if tuple(st["shape"]) != (self.B, self.H, self.cap_total, self.D) or list(st["segments"]) != \
+                list(self.segments) or list(st["caps"]) != list(self.caps) or \
+                not np.array_equal(np.asarray(st["lengths"]), self.lengths):
+            raise ValueError("the snapshot was taken on a window of another shape or layout")
+        self.__dict__.pop("_step_graphs", None)
+        for name in ("k_raw", "k_att", "v", "clock"):
+            getattr(self, name).copy_(st[name])
+        if "ring_ptr" in st:
+            self.pos = st["pos_loaded"].to(self.device)
+            self._ring_setup(int(st["slide_frames"]))
+            self._phase_tables()
+            if set(st["ring_ptr"]) != set(self.rings):
+                raise ValueError("the snapshot's rings do not match this window")
+            self.ring_ptr = {k: int(st["ring_ptr"][k]) for k in self.rings}
+            self.pos = self._phases[tuple(self.ring_ptr.values())]
+        else:
+            if hasattr(self, "rings"):
+                del self.rings
+            self.pos = torch.zeros_like(self.pos)
+            self.pos.copy_(st["pos"])
+        torch.cuda.synchronize(self.device)
+
 
 class HostStepPipeline:
     """Runs consecutive streaming steps for a caller that holds its tensors in

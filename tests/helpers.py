@@ -37,3 +37,15 @@ def sample_rows(n: int, k: int, seed: int) -> list:
     rng = np.random.default_rng(seed)
     extra = set(rng.choice(n, size=min(k, n), replace=False).tolist())
     return sorted(r for r in fixed | extra if 0 <= r < n)
+
+
+def assert_rope_close(got, ref, x):
+    """Within one bf16 ulp of the fp64 rotation, except where the rotated
+    component nearly cancels: there the fp32 rotation's own error (a few
+    2^-24 of the pair's norm) may exceed half an ulp of the tiny result, so
+    an absolute 2^-21 * |pair| is allowed.  x: the rotated input."""
+    ulps = ulp_diff_bf16(got, ref)
+    xd = x.double().numpy() if hasattr(x, "double") else np.asarray(x, dtype=np.float64)
+    pair = np.repeat(np.hypot(xd[..., 0::2], xd[..., 1::2]), 2, axis=-1)
+    err = np.abs(got.double().numpy() - ref)
+    assert np.all((ulps <= 1) | (err <= 2.0 ** -21 * pair))

@@ -11,7 +11,7 @@ def _line(ts, sm, reasons=("Not Active",) * 4):
 
 
 def test_clock_summary_keeps_the_timed_window():
-    t = time.time()
+    t = int(time.time()) + 0.25   # the stamps carry whole seconds + .250: keep t on that grid
     text = "\n".join([_line(t - 3, 600), _line(t - 1, 1800, ("Not Active", "Not Active", "Not Active", "Active")),
                       _line(t, 1700), _line(t + 5, 1965)])
     s = bench.ClockSampler.summarize(text, t - 1.5, t + 1)
@@ -29,6 +29,28 @@ def test_launch_count_follows_the_slide_plan():
     spec = workloads.scaled(workloads.CHUNK_TIERED, n_heads=1, head_dim=128, prompt_len=8, chunk_audio_tokens=4)
     win = StreamingWindow([spec], device="cpu")
     win._ring_setup(3)
-    # CPU window: no split workspace -> 4 launches per step (append, 2 RoPE, attention) + 3 for the slide
-    assert bench.launches_in_steps(win, True, 10) == 10 * (4 + 3)
+    # CPU window: no split workspace -> 4 launches per step (append, 2 RoPE, attention) + 4 for the slide
+    # (clock advance, two pooling boundaries, the clean-frame append)
+    assert bench.launches_in_steps(win, True, 10) == 10 * (4 + 4)
     assert bench.launches_in_steps(win, False, 10) == 40
+
+
+class _Ev:
+    def __init__(self, t):
+        self.t = t
+
+    def elapsed_time(self, other):
+        return other.t - self.t
+
+
+def test_call_breakdown_sums_split_calls_and_averages_steps():
+    e = [_Ev(x) for x in (0.0, 0.01, 0.03, 0.05, 0.55)]
+    step = [("pool a->b", 100, e[0], e[1]), ("pool a->b", 50, e[1], e[2]), ("rope", 300, e[2], e[3]),
+            ("attention", None, e[3], e[4])]
+    rows = {n: (ms, nb) for n, ms, nb in bench.call_breakdown([step, step])}
+    assert abs(rows["pool a->b"][0] - 0.03) < 1e-12 and rows["pool a->b"][1] == 150
+    assert abs(rows["attention"][0] - 0.5) < 1e-12
+    blk = bench.hbm_block(bench.call_breakdown([step]), 6556.0, "measured")
+    assert [r["call"] for r in blk["calls"]] == ["pool a->b", "rope"]          # attention is not HBM-bound
+    assert abs(blk["calls"][1]["achieved"] - 300 / 0.02e-3 / 1e9) < 1e-9
+    assert abs(blk["step_ms_sum_of_calls"] - 0.55) < 1e-12

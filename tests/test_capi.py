@@ -9,7 +9,8 @@ from streaming_video_audio_b200 import capi
 
 EXPECTED = {"sr_version", "sr_get_last_error", "sr_rope3d_apply", "sr_history_compress", "sr_kv_append",
             "sr_chunk_attention_fwd", "sr_chunk_attention_workspace_bytes", "sr_qknorm_rope3d_apply",
-            "sr_gather_tokens", "sr_gather_rope3d_tokens", "sr_scatter_tokens", "sr_chunk_attention_fwd_noalloc"}
+            "sr_gather_tokens", "sr_gather_rope3d_tokens", "sr_scatter_tokens", "sr_chunk_attention_fwd_noalloc",
+            "sr_set_wait_limit_ns", "sr_set_withheld_kv_tile", "sr_stream_clock_advance"}
 
 
 def test_header_declares_the_boundary():
@@ -51,27 +52,45 @@ def test_attention_rejects_bad_arguments_on_host():
 def test_rope_rejects_bad_arguments_on_host():
     lib = capi.load()
     cfg = capi.sr_rope_cfg(10000.0, 32, 48, 48)
-    call = lambda D=128, c=cfg, x=16, y=32, xs=(0, 5120, 128): lib.sr_rope3d_apply(
-        x, y, None, 1, 4, 40, D, None, c, 1.0, xs[0], xs[1], xs[2], 0, 5120, 128, 0, None)
+    call = lambda D=128, c=cfg, x=16, y=32, xs=(0, 5120, 128), t0=None: lib.sr_rope3d_apply(
+        x, y, None, 1, 4, 40, D, None, c, 1.0, xs[0], xs[1], xs[2], 0, 5120, 128, 0, t0, None)
     assert call(D=64) == capi.SR_ERR_INVALID_ARG                          # split does not sum to D
     assert call(c=capi.sr_rope_cfg(10000.0, 30, 50, 48)) == capi.SR_ERR_INVALID_ARG
     assert call(x=8) == capi.SR_ERR_INVALID_ARG                           # misaligned
     assert call(xs=(0, 5120, 100)) == capi.SR_ERR_INVALID_ARG             # stride not a multiple of 8
-    assert lib.sr_rope3d_apply(16, 32, None, 1, 0, 40, 128, None, cfg, 1.0, 0, 0, 0, 0, 0, 0, 0, None) == capi.SR_OK
+    assert call(t0=20) == capi.SR_ERR_INVALID_ARG and "t_origin" in _err(lib)   # clock not 8-byte aligned
+    assert lib.sr_rope3d_apply(16, 32, None, 1, 0, 40, 128, None, cfg, 1.0, 0, 0, 0, 0, 0, 0, 0, None,
+                               None) == capi.SR_OK
 
 
 def test_append_and_pool_reject_bad_arguments_on_host():
     lib = capi.load()
-    rc = lib.sr_kv_append(16, 32, None, 1, 2, 128, 256, 200, 48, 64, None, 100, None, 0, 256, 128, 0, None)
+    rc = lib.sr_kv_append(16, 32, None, 1, 2, 128, 256, 200, 48, 64, None, 100, None, 0, 256, 128, 0, None, None)
     assert rc == capi.SR_ERR_INVALID_ARG and "exceed" in _err(lib)
+    # a fused rotation needs positions and sub-blocks that sum to head_dim
+    rot = capi.sr_rope_out(80, None, 0, None, capi.sr_rope_cfg(10000.0, 32, 48, 48), 1.0)
+    rc = lib.sr_kv_append(None, 32, None, 1, 2, 128, 256, 0, 48, 64, None, 100, None, 0, 256, 128, 0,
+                          ctypes.byref(rot), None)
+    assert rc == capi.SR_ERR_INVALID_ARG and "positions" in _err(lib)
+    rot = capi.sr_rope_out(80, 96, 0, None, capi.sr_rope_cfg(10000.0, 32, 48, 40), 1.0)
+    rc = lib.sr_kv_append(None, 32, None, 1, 2, 128, 256, 0, 48, 64, None, 100, None, 0, 256, 128, 0,
+                          ctypes.byref(rot), None)
+    assert rc == capi.SR_ERR_INVALID_ARG and "sub-blocks" in _err(lib)
+    rc = lib.sr_kv_append(None, 32, None, 1, 2, 128, 256, 0, 48, 64, None, 100, None, 0, 256, 128, 0, None, None)
+    assert rc == capi.SR_ERR_INVALID_ARG and "without its buffer" in _err(lib)    # K with no buffer, no rotation
+    assert lib.sr_stream_clock_advance(None, 3.0, None) == capi.SR_ERR_INVALID_ARG
     cfg = capi.sr_pool_cfg(24, 42, 9, 2)
     rc = lib.sr_history_compress(16, 32, 48, 64, 1, 1, 2, 128, cfg, 0, 0, 256, 128, 0, 0, 256, 128,
-                                 None, None, 0, None, None)
+                                 None, None, 0, None, None, None)
     assert rc == capi.SR_ERR_INVALID_ARG
     cfg = capi.sr_pool_cfg(24, 42, 2, 2)
     rc = lib.sr_history_compress(16, None, 48, 64, 1, 1, 2, 128, cfg, 0, 0, 256, 128, 0, 0, 256, 128,
-                                 None, None, 0, None, None)
+                                 None, None, 0, None, None, None)
     assert rc == capi.SR_ERR_INVALID_ARG
+    rot = capi.sr_rope_out(88, 96, 0, None, capi.sr_rope_cfg(10000.0, 32, 48, 48), 1.0)   # k_rot misaligned
+    rc = lib.sr_history_compress(16, 32, 48, 64, 1, 1, 2, 128, cfg, 0, 0, 256, 128, 0, 0, 256, 128,
+                                 None, None, 0, None, ctypes.byref(rot), None)
+    assert rc == capi.SR_ERR_INVALID_ARG and "k_rot" in _err(lib)
 
 
 def test_gather_and_scatter_reject_bad_arguments_on_host():
@@ -80,7 +99,8 @@ def test_gather_and_scatter_reject_bad_arguments_on_host():
     # dst, src, idx, src_pos, B, S, H, D, cfg, scale, src_t, src_h, dst_b, dst_s, dst_h, stream
     def rope(dst=16, src=32, idx=48, pos=64, S=10, D=128, c=cfg, ts=512):
         # dst, src, idx, src_pos, B, S, H, D, cfg, scale, src_t, src_h, dst_b, dst_s, dst_h, stream
-        return lib.sr_gather_rope3d_tokens(dst, src, idx, pos, 2, S, 4, D, c, 1.0, ts, 128, 5120, 512, 128, None)
+        return lib.sr_gather_rope3d_tokens(dst, src, idx, pos, 2, S, 4, D, c, 1.0, ts, 128, 5120, 512, 128, None,
+                                           None)
 
     assert rope(pos=None) == capi.SR_ERR_INVALID_ARG and "src_pos" in _err(lib)
     assert rope(c=capi.sr_rope_cfg(10000.0, 32, 48, 40)) == capi.SR_ERR_INVALID_ARG
@@ -100,3 +120,10 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(capi, "_lib", None)
     with pytest.raises(RuntimeError, match="libsr.so not found"):
         capi.load()
+
+
+def test_failure_settings_validate_on_host():
+    lib = capi.load()
+    assert lib.sr_set_withheld_kv_tile(-2) == capi.SR_ERR_INVALID_ARG
+    assert lib.sr_set_withheld_kv_tile(-1) == capi.SR_OK
+    assert lib.sr_set_wait_limit_ns(0) == capi.SR_OK       # back to the default

@@ -11,7 +11,7 @@ import torch
 import oracle
 import workloads
 from streaming_video_audio_b200 import capi
-from tests.helpers import ATTN_MAX_ABS, ATTN_MEAN_ABS, LSE_ABS, attn_errors, ulp_diff_bf16
+from tests.helpers import ATTN_MAX_ABS, ATTN_MEAN_ABS, LSE_ABS, assert_rope_close, attn_errors, ulp_diff_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -19,17 +19,6 @@ DEV = "cuda"
 
 
 # ---------------------------------------------------------------- RoPE (a3)
-def assert_rope_close(got, ref, x):
-    """Within one bf16 ulp of the fp64 rotation, except where the rotated
-    component nearly cancels: there the fp32 rotation's own error (a few
-    2^-24 of the pair's norm) may exceed half an ulp of the tiny result, so
-    an absolute 2^-21 * |pair| is allowed."""
-    ulps = ulp_diff_bf16(got, ref)
-    xd = x.double().numpy()
-    pair = np.repeat(np.hypot(xd[..., 0::2], xd[..., 1::2]), 2, axis=-1)
-    err = np.abs(got.double().numpy() - ref)
-    assert np.all((ulps <= 1) | (err <= 2.0 ** -21 * pair))
-
 
 
 @pytest.mark.parametrize("D,split,H,N", [(128, (32, 48, 48), 40, 300), (64, (16, 24, 24), 3, 77),
@@ -139,6 +128,82 @@ def test_kv_append_exact_and_in_place():
         assert torch.equal(pb[b, 100:100 + n].cpu(), ps[b, :n])
         assert not kb[b, :, :100].any() and not kb[b, :, 100 + n:].any()
         assert not pb[b, 100 + n:].any()
+
+
+@pytest.mark.parametrize("with_raw", [True, False])
+def test_kv_append_with_fused_rotation(with_raw):
+    """The cache write and the RoPE in one pass: K lands rotated in k_rot at
+    its position plus the stream clock (t_origin), optionally also unrotated
+    in k_buf (bit-exact copy), V is copied bit-exactly; slots outside
+    [dst, dst + n_valid) stay untouched."""
+    B, H, D, cap, N, dst = 2, 40, 128, 512, 200, 128
+    split = (32, 48, 48)
+    kb = torch.zeros(B, H, cap, D, dtype=torch.bfloat16, device=DEV)
+    kr = torch.zeros_like(kb)
+    vb = torch.zeros_like(kb)
+    ks = workloads.draw_tensor((B, N, H, D), seed=17)
+    vs = workloads.draw_tensor((B, N, H, D), seed=18)
+    ps = torch.stack([workloads.draw_positions(N, seed=19), workloads.draw_positions(N, seed=20)])
+    clock = torch.tensor([1234.0], dtype=torch.float64, device=DEV)
+    nv = torch.tensor([N, 150], dtype=torch.int32, device=DEV)
+    rot = capi.RopeOut(kr, ps.to(DEV), split, t_origin=clock)
+    capi.sr_kv_append(kb if with_raw else None, vb, None, dst, ks.to(DEV), vs.to(DEV), None, n_valid=nv, rot=rot)
+    torch.cuda.synchronize()
+    for b, n in enumerate((N, 150)):
+        shifted = ps[b, :n].double().numpy() + np.array([1234.0, 0.0, 0.0])
+        ref = oracle.rope3d(ks[b, :n], shifted, split)
+        assert_rope_close(kr[b, :, dst:dst + n].permute(1, 0, 2).cpu(), ref, ks[b, :n])
+        assert torch.equal(vb[b, :, dst:dst + n].cpu(), vs[b, :n].permute(1, 0, 2))
+        if with_raw:
+            assert torch.equal(kb[b, :, dst:dst + n].cpu(), ks[b, :n].permute(1, 0, 2))
+        else:
+            assert not kb.any()
+        for t in (kr, vb):
+            assert not t[b, :, :dst].any() and not t[b, :, dst + n:].any()
+
+
+def test_history_compress_with_fused_rotation():
+    """Pooling with the pooled key rotated on its way into the tier: k_rot
+    equals the RoPE (at the given cell positions plus the clock) of the
+    pooled bf16 key k_out holds."""
+    gh, gw, ph, pw, B, F, H, D = 24, 42, 2, 2, 1, 3, 40, 128
+    split = (32, 48, 48)
+    cells = 12 * 21
+    k = workloads.draw_tensor((B, F, gh * gw, H, D), seed=24)
+    v = workloads.draw_tensor((B, F, gh * gw, H, D), seed=25)
+    ko = torch.zeros(B, F, cells, H, D, dtype=torch.bfloat16, device=DEV)
+    vo, kr = torch.zeros_like(ko), torch.zeros_like(ko)
+    rpos = torch.stack([workloads.draw_positions(F * cells, seed=26)]).to(DEV)
+    clock = torch.tensor([-57.0], dtype=torch.float64, device=DEV)
+    capi.sr_history_compress(k.to(DEV), v.to(DEV), ko, vo, (gh, gw), (ph, pw),
+                             rot=capi.RopeOut(kr, rpos, split, t_origin=clock))
+    torch.cuda.synchronize()
+    pooled = ko[0].reshape(F * cells, H, D).cpu()
+    ref = oracle.rope3d(pooled, rpos[0].double().cpu().numpy() + np.array([-57.0, 0.0, 0.0]), split)
+    assert_rope_close(kr[0].reshape(F * cells, H, D).cpu(), ref, pooled)
+    ref_v = oracle.pool(v[0].reshape(F, gh, gw, H, D), ph, pw).reshape(F, cells, H, D)
+    assert ulp_diff_bf16(vo[0].cpu(), ref_v).max() <= 1
+
+
+def test_rope_t_origin_and_stream_clock():
+    """t_origin adds the stream clock to every t (formed in fp64): the result
+    matches the oracle's rotation at the shifted positions; the clock kernel
+    adds exactly."""
+    B, N, H, D = 1, 64, 8, 128
+    split = (32, 48, 48)
+    x = workloads.draw_tensor((B, N, H, D), seed=33)
+    pos = workloads.draw_positions(N, seed=34)[None]
+    clock = torch.zeros(1, dtype=torch.float64, device=DEV)
+    for _ in range(7):
+        capi.sr_stream_clock_advance(clock, 3.0)
+    capi.sr_stream_clock_advance(clock, 0.5)
+    torch.cuda.synchronize()
+    assert float(clock.item()) == 21.5
+    y = torch.zeros(B, H, N, D, dtype=torch.bfloat16, device=DEV)
+    capi.sr_rope3d_apply(x.to(DEV), y.permute(0, 2, 1, 3), pos.to(DEV), split, t_origin=clock)
+    torch.cuda.synchronize()
+    ref = oracle.rope3d(x[0], pos[0].double().numpy() + np.array([21.5, 0.0, 0.0]), split)
+    assert_rope_close(y[0].permute(1, 0, 2).cpu(), ref, x[0])
 
 
 # ---------------------------------------------------------------- attention (a4)
@@ -274,6 +339,71 @@ def test_attention_repeated_launches_deterministic():
     for _ in range(10):
         o, l = _run_attention(q, k, v, caps, lens, q_len, use_workspace=False)
         assert torch.equal(o[0, :129], _run_attention(q, k, v, caps, lens, q_len, use_workspace=False)[0][0, :129])
+
+
+@pytest.mark.parametrize("use_workspace", [True, False])
+def test_attention_q_len_past_q_cap_writes_inside_buffers(use_workspace):
+    """A device q_len larger than q_cap (the host cannot see it) is clamped in
+    the kernels: rows [0, q_cap) are computed as for q_len = q_cap and guard
+    memory after o and lse keeps its sentinel.  q_cap = 300 is not a multiple
+    of the 256-row query block, so the last block reaches past the buffer."""
+    D, H, caps, lens, q_cap = 128, 2, [256, 512], [[256, 400]], 300
+    q, k, v = _draw_case(D, H, caps, lens, [q_cap], seed=45)
+    guard = 300
+    o_full = torch.full((q_cap + guard, H, D), 7.0, dtype=torch.bfloat16, device=DEV)
+    lse_full = torch.full((H * q_cap + 2 * guard,), 7.0, dtype=torch.float32, device=DEV)
+    o, lse = o_full[:q_cap].view(1, q_cap, H, D), lse_full[:H * q_cap].view(1, H, q_cap)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    nbytes = capi.sr_chunk_attention_workspace_bytes(1, H, D, q_cap)
+    assert nbytes > 0
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=DEV) if use_workspace else None
+    capi.sr_chunk_attention_fwd(q.to(DEV).contiguous(), k.to(DEV).contiguous(), v.to(DEV).contiguous(), o, lse,
+                                caps, torch.tensor(lens, dtype=torch.int32, device=DEV),
+                                torch.tensor([q_cap + 100], dtype=torch.int32, device=DEV), 1 / math.sqrt(D),
+                                status, workspace=ws)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert torch.all(o_full[q_cap:] == 7.0) and torch.all(lse_full[H * q_cap:] == 7.0)
+    for h in range(H):
+        kk, vv = _valid_kv(k, v, 0, h, caps, lens[0])
+        ro, rl = oracle.attention(q[0, h], kk, vv, 1 / math.sqrt(D))
+        mx, mean = attn_errors(o[0, :, h].cpu(), ro)
+        assert mx <= ATTN_MAX_ABS and mean <= ATTN_MEAN_ABS, (h, mx, mean)
+        assert np.abs(lse[0, h].double().cpu().numpy() - rl).max() <= LSE_ABS
+
+
+@pytest.mark.parametrize("D", [128, 64])
+def test_attention_wait_runs_out_reports_timeout_and_context_survives(D):
+    """Failure detection without a GPU fault: with the load of K tile 1
+    withheld (the library's test hook) and a 2 ms wait limit, the pipeline
+    wait for that tile runs out; the launch writes SR_ERR_DEVICE_TIMEOUT into
+    the status word, waits for its own loads and MMAs in flight, releases its
+    tensor memory and returns.  The context stays usable: the next normal
+    launch matches the oracle."""
+    H, caps, lens, q_len = 2, [256, 512], [[200, 400]], [300]
+    q, k, v = _draw_case(D, H, caps, lens, q_len, seed=47)
+    qd, kd, vd = (t.to(DEV).contiguous() for t in (q, k, v))
+    kl = torch.tensor(lens, dtype=torch.int32, device=DEV)
+    ql = torch.tensor(q_len, dtype=torch.int32, device=DEV)
+    o = torch.zeros(1, 300, H, D, dtype=torch.bfloat16, device=DEV)
+    lse = torch.zeros(1, H, 300, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    capi.sr_set_wait_limit_ns(2_000_000)
+    capi.sr_set_withheld_kv_tile(1)
+    try:
+        # whole units (no workspace): every work item walks all 6 KV tiles
+        capi.sr_chunk_attention_fwd(qd, kd, vd, o, lse, caps, kl, ql, 1 / math.sqrt(D), status, workspace=None)
+        torch.cuda.synchronize()
+    finally:
+        capi.sr_set_withheld_kv_tile(-1)
+        capi.sr_set_wait_limit_ns(0)
+    assert int(status.item()) == capi.SR_ERR_DEVICE_TIMEOUT
+    o2, l2 = _run_attention(q, k, v, caps, lens, q_len)
+    for h in range(H):
+        kk, vv = _valid_kv(k, v, 0, h, caps, lens[0])
+        ro, rl = oracle.attention(q[0, h, :300], kk, vv, 1 / math.sqrt(D))
+        mx, mean = attn_errors(o2[0, :300, h], ro)
+        assert mx <= ATTN_MAX_ABS and mean <= ATTN_MEAN_ABS, (h, mx, mean)
 
 
 # ---------------------------------------------------------------- QK-norm + RoPE (fused)
