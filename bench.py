@@ -318,6 +318,36 @@ def oracle_sample(spec, inp, target_s: float, heads=None):
     return fl / dt / 1e12, rows, dt, o
 
 
+def torch_sdpa_context(win, flops: float, n: int):
+    """Context only, not a product path: torch's scaled_dot_product_attention
+    (the backend torch picks among cuDNN, flash and memory-efficient) on the
+    same rotated queries and the valid rotated keys and values of the
+    window, gathered into dense tensors once, timed like the library's
+    attention.  Returns its TFLOP/s and ms, or the reason it could not run."""
+    try:
+        from torch.nn.attention import SDPBackend, sdpa_kernel
+        idx = torch.from_numpy(np.nonzero(win.valid_mask(0))[0]).to(win.device)
+        lq = int(win.q_len[0].item())
+        q = win.q_att[:, :, :lq].contiguous()
+        k = win.k_att.index_select(2, idx).contiguous()
+        v = win.v.index_select(2, idx).contiguous()
+        backends = [SDPBackend.CUDNN_ATTENTION, SDPBackend.FLASH_ATTENTION, SDPBackend.EFFICIENT_ATTENTION]
+        with sdpa_kernel(backends, set_priority=True):
+            for _ in range(3):
+                torch.nn.functional.scaled_dot_product_attention(q, k, v, scale=win.scale)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(n):
+                torch.nn.functional.scaled_dot_product_attention(q, k, v, scale=win.scale)
+            e1.record()
+            torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / n
+        return {"ms": ms, "tflops": flops / (ms * 1e-3) / 1e12,
+                "note": "torch SDPA, backend chosen by torch (cuDNN, flash or memory-efficient); context only"}
+    except Exception as exc:   # context only: never fails the bench
+        return {"unavailable": f"{type(exc).__name__}: {exc}"[:200]}
+
+
 def run_configs(main_config: int, device, peak: float, n_attn: int = 20, target_s: float = 6.0,
                 others_s: float = 2.0):
     """Every workload config once, after the timed region: a fresh window on
@@ -361,6 +391,7 @@ def run_configs(main_config: int, device, peak: float, n_attn: int = 20, target_
         win.check_status()
         attn_ms = ev[0].elapsed_time(ev[1]) / n_attn
         flops = attention_flops(specs)
+        sdpa = torch_sdpa_context(win, flops, n_attn) if win.B == 1 else None
         spec, inp = specs[0], inputs[0]
         heads = None if c in (1, 2, 3) else [0, spec.n_heads // 2]
         val, rows, dt, ref = oracle_sample(spec, inp, target_s if c == main_config else others_s, heads=heads)
@@ -372,6 +403,7 @@ def run_configs(main_config: int, device, peak: float, n_attn: int = 20, target_
             "frac_of_burst": flops / (attn_ms * 1e-3) / 1e12 / peak,
             "parity": {"max_abs": float(err.max()), "mean_abs": float(err.mean()), "rows": len(rows),
                        "heads": len(sel), "session": 0, "bar": [2e-2, 2e-3]},
+            "torch_sdpa_context": sdpa,
             "oracle": {"value": val, "unit": "TFLOP/s", "rows": len(rows), "heads": len(sel), "seconds": dt}}
         del win, chunk, o_gpu
         torch.cuda.empty_cache()

@@ -349,7 +349,7 @@ int sr_stream_clock_advance(double *clock_dev, double frames, void *stream) {
 
 size_t sr_chunk_attention_workspace_bytes(int32_t n_batch, int32_t n_heads, int32_t head_dim, int32_t q_cap) {
     if (n_batch < 1 || n_heads < 1 || q_cap < 1 || (head_dim != 64 && head_dim != 128)) return 0;
-    return attention_schedule(n_batch, n_heads, head_dim, q_cap, attention_slots(head_dim)).workspace_bytes;
+    return attention_schedule(n_batch, n_heads, head_dim, q_cap, attention_sm_count()).workspace_bytes;
 }
 
 int sr_chunk_attention_fwd(const void *q, const void *k, const void *v, void *o, float *lse,

@@ -1,8 +1,5 @@
 // chunk_attention.cu -- fused chunk attention over [prompt | context | chunk]
-// KV segments on sm_100a (tcgen05 tensor cores, TMEM accumulators, TMA): the
-// dispatch of sr_chunk_attention_fwd, the split-KV work list and merge, and
-// the single-SM kernel used at head_dim 64 (head_dim 128 runs on CTA pairs,
-// pair_attention.cu).
+// KV segments on sm_100a (tcgen05 tensor cores, TMEM accumulators, TMA).
 //
 // What it computes (plain definition, no causal mask): for every valid query
 // row i of a (session, head),
@@ -127,8 +124,8 @@ struct TileWalk {
 
 
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                          int32_t *status, uint64_t limit) {
-    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, status, limit));
+                                          int32_t *status, uint64_t limit, uint32_t suspend_ns = 0) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, status, limit, suspend_ns));
 }
 
 template <int D>
@@ -344,8 +341,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     continue;
                 }
                 if (!ok) break;
-                if (!(ok = warp_wait(&stats_ready[t], 0, abort_flag, p.status, limit))) break;
-                if (!(ok = warp_wait(&o_done[t], (n_tiles - 1) & 1, abort_flag, p.status, limit))) break;
+                if (!(ok = warp_wait(&stats_ready[t], 0, abort_flag, p.status, limit, 20000u))) break;
+                if (!(ok = warp_wait(&o_done[t], (n_tiles - 1) & 1, abort_flag, p.status, limit, 20000u))) break;
                 tc_fence_after();
                 const float l_row = row_l[t * kTileM + row];
                 const float inv_l = 1.0f / l_row;
@@ -500,15 +497,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int st = j % kStages;
                     const int st1 = (j + 1) % kStages;
                     const bool more = j + 1 < n_tiles;
+                    // load waits first (the tiles landed long ago): once P arrives, the
+                    // MMAs follow each other without a wait that would idle the pipe
                     if (!(ok = mbar_wait(&v_full[st], (j / kStages) & 1, abort_flag, p.status, limit))) break;
+                    if (more && !(ok = mbar_wait(&k_full[st1], ((j + 1) / kStages) & 1, abort_flag, p.status, limit)))
+                        break;
                     if (!(ok = mbar_wait(&p_full[0], j & 1, abort_flag, p.status, limit))) break;
                     tc_fence_after();
                     issue_pv(0, st, j > 0);
-                    if (more) {
-                        if (!(ok = mbar_wait(&k_full[st1], ((j + 1) / kStages) & 1, abort_flag, p.status, limit))) break;
-                        tc_fence_after();
-                        issue_qk(0, st1);
-                    }
+                    if (more) issue_qk(0, st1);
                     if (!(ok = mbar_wait(&p_full[1], j & 1, abort_flag, p.status, limit))) break;
                     tc_fence_after();
                     issue_pv(1, st, j > 0);
@@ -713,11 +710,8 @@ AttnSchedule attention_schedule(int32_t n_batch, int32_t n_heads, int32_t head_d
 
 int attention_sm_count() { return sm_count(); }
 
-int attention_slots(int32_t head_dim) { return head_dim == 128 ? attention_pair_slots() : sm_count(); }
-
 int launch_chunk_attention(const AttnLaunch &a) {
-    if (a.head_dim == 128)
-        return launch_pair_attention(a, attention_schedule(a.n_batch, a.n_heads, 128, a.q_cap, attention_pair_slots()));
+    if (a.head_dim == 128) return launch<128>(a);
     if (a.head_dim == 64) return launch<64>(a);
     return set_error(SR_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
 }

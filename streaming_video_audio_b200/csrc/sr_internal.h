@@ -54,10 +54,6 @@ struct AttnSchedule {
 };
 AttnSchedule attention_schedule(int32_t n_batch, int32_t n_heads, int32_t head_dim, int32_t q_cap, int32_t sms);
 int attention_sm_count();
-// Units that run at once: CTA pairs at head_dim 128 (pair kernel), SMs at 64.
-int attention_slots(int32_t head_dim);
-int attention_pair_slots();
-int launch_pair_attention(const AttnLaunch &a, const AttnSchedule &sc);
 // Merge of the KV parts of split units (fp32 partials in the workspace).
 int launch_split_combine(const float *ws_o, const float *ws_ml, void *o, float *lse, const int32_t *q_len,
                          int32_t n_full, int32_t split, int32_t tail_units, int32_t qb_per_head, int32_t n_heads,
