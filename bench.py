@@ -192,10 +192,10 @@ def build_window(config: int, rank: int, device):
     return specs, inputs, win, chunk
 
 
-# sources of the attention launch at head_dim 128 (pair kernel, dispatch and
-# split merge, device helpers): a traffic record is only used while they are
-# unchanged since its capture
-ATTENTION_SOURCES = ("pair_attention.cu", "chunk_attention.cu", "sr_device.cuh")
+# sources of the attention launch (kernel, dispatch and split merge, device
+# helpers): a traffic record is only used while they are unchanged since its
+# capture
+ATTENTION_SOURCES = ("chunk_attention.cu", "sr_device.cuh")
 
 
 def attention_source_hash() -> str:
