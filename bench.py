@@ -41,6 +41,7 @@ import statistics
 import subprocess
 import sys
 import tempfile
+import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -92,29 +93,66 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms; mark()
-    brackets the timed region on the host clock, and stop() keeps the samples
-    taken inside it (all samples, flagged, when the region was too short to
-    catch one)."""
+    """SM clocks and throttle reasons of the timed GPU, sampled while the
+    timed region runs; mark() brackets that region on the host clock, and
+    stop() keeps the samples taken inside it (all samples, flagged, when none
+    fell inside).  NVML is polled every 2 ms from a thread (a 20-step region
+    lasts only ~14 ms); without NVML, nvidia-smi samples every 200 ms."""
     FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASON_BITS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+                   "sw_power_cap": 0x4}
 
-    def __init__(self, gpu_index: int):
-        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+    def __init__(self, device: int):
         self.window = [None, None]
+        self.p = None
+        self.thread = None
+        self.samples = []
         try:
-            self.p = subprocess.Popen(["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}",
-                                       "--format=csv,noheader,nounits", "-lms", "200"],
-                                      stdout=self.f, stderr=subprocess.DEVNULL)
-        except OSError:
-            self.p = None
+            import pynvml
+            pynvml.nvmlInit()
+            pr = torch.cuda.get_device_properties(device)
+            h = pynvml.nvmlDeviceGetHandleByPciBusId(
+                f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0")
+            self.done = threading.Event()
+
+            def poll():
+                while not self.done.is_set():
+                    try:
+                        self.samples.append((time.time(), pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
+                                             pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM),
+                                             pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)))
+                    except pynvml.NVMLError:
+                        return
+                    time.sleep(0.002)
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.thread = None
+            self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            try:
+                self.p = subprocess.Popen(["nvidia-smi", "-i", self.smi_index(device), f"--query-gpu={self.FIELDS}",
+                                           "--format=csv,noheader,nounits", "-lms", "200"],
+                                          stdout=self.f, stderr=subprocess.DEVNULL)
+            except OSError:
+                self.p = None
         time.sleep(0.3)
+
+    @staticmethod
+    def smi_index(device: int) -> str:
+        """nvidia-smi's id of CUDA device `device` (CUDA_VISIBLE_DEVICES maps it)."""
+        vis = [v.strip() for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+        return vis[device] if device < len(vis) else str(device)
 
     def mark(self, i: int) -> None:
         self.window[i] = time.time()
 
     def stop(self):
+        if self.thread is not None:
+            self.done.set()
+            self.thread.join(timeout=5)
+            return self.summarize_samples(self.samples, *self.window)
         if self.p is None:
             return None
         self.p.terminate()
@@ -126,6 +164,24 @@ class ClockSampler:
         text = open(self.f.name).read()
         os.unlink(self.f.name)
         return self.summarize(text, *self.window)
+
+    @classmethod
+    def summarize_samples(cls, samples, t0=None, t1=None):
+        """The same summary from NVML samples (time, sm MHz, max MHz, reason bits)."""
+        rows = [(ts, float(sm), float(mx), {n for n, bit in cls.REASON_BITS.items() if r & bit})
+                for ts, sm, mx, r in samples]
+        return cls._summary(rows, t0, t1, "nvml, 2 ms")
+
+    @staticmethod
+    def _summary(samples, t0, t1, source):
+        if not samples:
+            return None
+        inside = [x for x in samples if t0 is not None and t1 is not None and t0 <= x[0] <= t1]
+        use = inside or samples
+        reasons = set().union(*[x[3] for x in use])
+        return {"sm_mhz": statistics.median(x[1] for x in use), "sm_max_mhz": use[-1][2],
+                "reasons": sorted(reasons), "samples": len(use), "in_timed_region": bool(inside),
+                "source": source}
 
     @staticmethod
     def summarize(text: str, t0=None, t1=None):
@@ -143,13 +199,7 @@ class ClockSampler:
                                 {n for n, v in zip(names, r[6:10]) if v.strip().lower() == "active"}))
             except (ValueError, IndexError):
                 continue
-        if not samples:
-            return None
-        inside = [x for x in samples if t0 is not None and t1 is not None and t0 <= x[0] <= t1]
-        use = inside or samples
-        reasons = set().union(*[x[3] for x in use])
-        return {"sm_mhz": statistics.median(x[1] for x in use), "sm_max_mhz": use[-1][2],
-                "reasons": sorted(reasons), "samples": len(use), "in_timed_region": bool(inside)}
+        return ClockSampler._summary(samples, t0, t1, "nvidia-smi, 200 ms")
 
 
 def rank_sessions(config: int, rank: int):

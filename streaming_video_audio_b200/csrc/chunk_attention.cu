@@ -61,27 +61,6 @@ constexpr int kPanelBytes = 128 * 128;   // 128 rows x 128 bytes (64 bf16), one 
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
-// Tuning switches (the values built by default were chosen by measurement).
-#ifndef SR_SPLIT_P_STORE
-#define SR_SPLIT_P_STORE 0
-#endif
-#ifndef SR_EXP2_FMA_EVERY
-#define SR_EXP2_FMA_EVERY 0
-#endif
-#ifndef SR_SOFTMAX_2PASS
-#define SR_SOFTMAX_2PASS 0
-#endif
-#ifndef SR_P_SPLIT_ARRIVE
-#define SR_P_SPLIT_ARRIVE 0
-#endif
-// store P's first 64 keys before the second half's exponentials
-constexpr bool kSplitPStore = SR_SPLIT_P_STORE != 0;
-// every kExpFmaEvery-th column's exponential on the FMA pipe (exp2_fma)
-// instead of the MUFU pipe; 0 = all on MUFU
-constexpr int kExpFmaEvery = SR_EXP2_FMA_EVERY;
-// hand P to the MMA issuer in two halves of 64 keys (p_lo, then p_full): the
-// PV of the first half runs while the second half is packed and stored
-constexpr bool kPSplit = SR_P_SPLIT_ARRIVE != 0 && SR_SOFTMAX_2PASS == 0;
 
 // Registers per thread after reallocation (launch: 65536 / 512 = 128 each):
 // 2 x 128 x 160 + 128 x 88 + 128 x 104 = 65536 (the launch total; no spills).
@@ -123,8 +102,8 @@ struct Smem {
     static constexpr int kV = kK + kStages * kTileBytes;
     static constexpr int kBar = kV + kStages * kTileBytes;
     // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S],
-    // s_full[2], p_full[2], o_done[2], stats_ready[2], drain, p_lo[2]
-    static constexpr int kNumBars = 1 + 4 * kStages + 5 * kQTiles + 1;
+    // s_full[2], p_full[2], o_done[2], stats_ready[2], drain
+    static constexpr int kNumBars = 1 + 4 * kStages + 4 * kQTiles + 1;
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kRow = kMisc + 16 + 12 * SR_MAX_SEG + 16;   // float l[2][128], m[2][128]
     static constexpr int kEnd = kRow + 2 * kQTiles * kTileM * 4;
@@ -188,7 +167,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *o_done = p_full + kQTiles;         // [2] MMA (PV_t) -> epilogue
     uint64_t *stats_ready = o_done + kQTiles;    // [2] softmax t -> epilogue: final row max / sum
     uint64_t *drain = stats_ready + kQTiles;     // every MMA issued so far is complete
-    uint64_t *p_lo = drain + 1;                  // [2] softmax t -> MMA: P_t keys [0, 64) (split hand-off)
     // Every waiter consumes each phase of its barrier in order, so parity
     // waits never alias: a barrier is never more than one phase ahead of the
     // phase its waiter asks for.
@@ -215,7 +193,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < kQTiles; ++t) {
             mbar_init(&s_full[t], 1);
             mbar_init(&p_full[t], 4);        // the four softmax warps of tile t
-            mbar_init(&p_lo[t], 4);
             mbar_init(&o_done[t], 1);
             mbar_init(&stats_ready[t], 4);
         }
@@ -289,68 +266,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int valid = min(kTileN, seg_len[w.s] - w.t * kTileN);
             if (!(ok = warp_wait(&s_full[t], j & 1, abort_flag, p.status, limit))) break;
             tc_fence_after();
-#if SR_SOFTMAX_2PASS
-            // Two passes over S in TMEM, 32 columns at a time, so that no more
-            // than 64 S values are live in registers: pass 1 takes the row max,
-            // pass 2 re-reads each chunk, forms its exponentials and stores its
-            // P right away (P chunk k overwrites S columns [16k, 16k + 16), all
-            // in chunks <= k, already read), the next chunk's load in flight.
-            float mx8[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-                uint32_t r[2][32];
-                tmem_ld32(s_addr + h2 * 64, r[0]);
-                tmem_ld32(s_addr + h2 * 64 + 32, r[1]);
-                tmem_wait_ld();
-#pragma unroll
-                for (int c = 0; c < 2; ++c)
-#pragma unroll
-                    for (int e = 0; e < 32; e += 16)
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const int col = h2 * 64 + c * 32 + e + i;
-                            const float a = col < valid ? __uint_as_float(r[c][e + i]) : -INFINITY;
-                            const float b2 = col + 8 < valid ? __uint_as_float(r[c][e + 8 + i]) : -INFINITY;
-                            mx8[i] = fmax3(mx8[i], a, b2);
-                        }
-            }
-            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-            const float m_new = fmaxf(m_run, mx * sl2);
-            const bool need = m_new > m_run + kRescaleThreshold;
-            const float m_use = need ? m_new : m_run;
-            const float alpha = need ? fast_exp2(m_run - m_use) : 1.0f;
-            float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            uint32_t r[2][32];
-            tmem_ld32(s_addr, r[0]);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                tmem_wait_ld();
-                if (c + 1 < 4) tmem_ld32(s_addr + (c + 1) * 32, r[(c + 1) & 1]);
-                uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    float x2[2];
-#pragma unroll
-                    for (int k = 0; k < 2; ++k) {
-                        const int col = c * 32 + 2 * e + k;
-                        const float v =
-                            col < valid ? fmaf(__uint_as_float(r[c & 1][2 * e + k]), sl2, -m_use) : -INFINITY;
-                        x2[k] = (kExpFmaEvery > 0 && col % (kExpFmaEvery > 0 ? kExpFmaEvery : 1) == kExpFmaEvery - 1)
-                                    ? exp2_fma(v)
-                                    : fast_exp2(v);
-                        sum8[(2 * e + k) & 7] += x2[k];
-                    }
-                    pk[e] = pack_bf16x2(x2[0], x2[1]);
-                }
-                tmem_st16(s_addr + c * 16, pk);
-            }
-            const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
-            l_run = l_run * alpha + sum;
-            m_run = m_use;
-#else
             float s[kTileN];
             {
                 uint32_t r[4][32];
@@ -380,54 +295,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool need = m_new > m_run + kRescaleThreshold;
             const float m_use = need ? m_new : m_run;
             const float alpha = need ? fast_exp2(m_run - m_use) : 1.0f;
-            // exponentials and P (bf16 pairs, over the first 64 columns of S_t) in
-            // two halves of 64 keys: the first half's TMEM store is under way
-            // while the second half's exponentials run
+            // exponentials, their row sum (eight partial sums), P as bf16 pairs
+            // over the first 64 columns of S_t
             float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-#pragma unroll
-                for (int c = half * 64; c < half * 64 + 64; ++c) {
-                    const float x = fmaf(s[c], sl2, -m_use);
-                    s[c] = (kExpFmaEvery > 0 && c % (kExpFmaEvery > 0 ? kExpFmaEvery : 1) == kExpFmaEvery - 1)
-                               ? exp2_fma(x)
-                               : fast_exp2(x);
-                    sum8[c & 7] += s[c];
-                }
-                if (kSplitPStore || (kPSplit && half == 0)) {
-                    uint32_t pk[32];
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(s[half * 64 + 2 * e], s[half * 64 + 2 * e + 1]);
-                    tmem_st32(s_addr + half * 32, pk);
-                }
-            }
-            if (kPSplit) {
-                // O_t's rescale (below) moves ahead of the first hand-off: PV of
-                // the first 64 keys already accumulates into O_t
-                if (j > 0 && __any_sync(0xffffffffu, need)) rescale_o(alpha);
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&p_lo[t]);
-                uint32_t pk[32];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(s[64 + 2 * e], s[64 + 2 * e + 1]);
-                tmem_st32(s_addr + 32, pk);
+            for (int c = 0; c < kTileN; ++c) {
+                s[c] = fast_exp2(fmaf(s[c], sl2, -m_use));
+                sum8[c & 7] += s[c];
             }
             const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
             l_run = l_run * alpha + sum;
             m_run = m_use;
-            if (!kSplitPStore && !kPSplit) {
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t pk[32];
+            for (int half = 0; half < 2; ++half) {
+                uint32_t pk[32];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(s[half * 64 + 2 * e], s[half * 64 + 2 * e + 1]);
-                    tmem_st32(s_addr + half * 32, pk);
-                }
+                for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(s[half * 64 + 2 * e], s[half * 64 + 2 * e + 1]);
+                tmem_st32(s_addr + half * 32, pk);
             }
-#endif
-            if (!kPSplit && j > 0 && __any_sync(0xffffffffu, need)) rescale_o(alpha);
+            if (j > 0 && __any_sync(0xffffffffu, need)) rescale_o(alpha);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -594,29 +480,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     umma_commit(&s_full[t]);
                 };
-                // O_t += P_t V over keys [16 kk0, 16 kk1) of the tile
-                auto issue_pv = [&](int t, int st, bool acc, int kk0, int kk1, bool last) {
+                auto issue_pv = [&](int t, int st, bool acc, bool last) {
                     const uint64_t b0 = umma_desc_advance(desc_v, st * L::kTileBytes);
                     const uint32_t d = tmem + tmem_o(t);
                     const uint32_t a = tmem + tmem_s(t);
 #pragma unroll
                     for (int kk = 0; kk < kTileN / 16; ++kk)
-                        if (kk >= kk0 && kk < kk1)
-                            umma_bf16_ts(d, a + kk * 8, umma_desc_advance(b0, kk * 2048), idesc_pv,
-                                         (acc || kk > 0) ? 1u : 0u);
+                        umma_bf16_ts(d, a + kk * 8, umma_desc_advance(b0, kk * 2048), idesc_pv,
+                                     (acc || kk > 0) ? 1u : 0u);
                     if (last) umma_commit(&o_done[t]);   // the epilogue reads only the final O
                 };
-                // P_t(j) -> O_t: whole, or in the two halves the softmax hands over
+                // P_t(j) -> O_t once the softmax of tile t has handed P_t(j) over
                 auto pv_step = [&](int t, int st, int j, bool last) -> bool {
-                    constexpr int kHalf = kTileN / 32;
-                    if (kPSplit) {
-                        if (!mbar_wait(&p_lo[t], j & 1, abort_flag, p.status, limit)) return false;
-                        tc_fence_after();
-                        issue_pv(t, st, j > 0, 0, kHalf, false);
-                    }
                     if (!mbar_wait(&p_full[t], j & 1, abort_flag, p.status, limit)) return false;
                     tc_fence_after();
-                    issue_pv(t, st, j > 0, kPSplit ? kHalf : 0, 2 * kHalf, last);
+                    issue_pv(t, st, j > 0, last);
                     return true;
                 };
                 bool ok = mbar_wait(q_full, 0, abort_flag, p.status, limit) &&

@@ -249,16 +249,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
-// 32 lanes x 16 consecutive 32-bit columns.
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-        : "memory");
-}
-
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -267,27 +257,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
-}
-
-// 2^x without the MUFU pipe (FMA and integer pipes only), for a share of a
-// softmax's exponentials so that the MUFU pipe is not the bottleneck:
-//   j = round(x): adding 1.5 * 2^23 leaves round(x) in the low mantissa bits
-//       of t (round to nearest), and t - 1.5 * 2^23 is that integer;
-//   2^f for f = x - j in [-1/2, 1/2] by a degree-3 polynomial (relative
-//       error 2^-13.7 < the 2^-9 of the bf16 weight it becomes; coefficients
-//       fitted to 2^f by an iteratively reweighted least-squares minimax fit);
-//   the exponent field gets j by one integer multiply-add: t's bits times 2^23
-//       are j << 23 modulo 2^32 (the bits of 1.5 * 2^23 shift out).
-// Valid for x in (-126, 127); x <= -126 (including -inf) returns 0.
-__device__ __forceinline__ float exp2_fma(float x) {
-    const float t = x + 12582912.0f;
-    const float j = t - 12582912.0f;
-    const float f = x - j;
-    float p = fmaf(f, 0.0551665202f, 0.242605433f);
-    p = fmaf(p, f, 0.693261445f);
-    p = fmaf(p, f, 0.999928474f);
-    const float r = __uint_as_float(__float_as_uint(t) * 8388608u + __float_as_uint(p));
-    return x > -126.0f ? r : 0.0f;
 }
 
 // max(a, b, c) in one instruction.
@@ -302,9 +271,5 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-__device__ __forceinline__ void st_shared_v4(uint32_t saddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(a), "r"(b), "r"(c), "r"(d)
-                 : "memory");
-}
 
 }  // namespace sr

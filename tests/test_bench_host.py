@@ -23,6 +23,18 @@ def test_clock_summary_keeps_the_timed_window():
     assert bench.ClockSampler.summarize("garbage line\n") is None
 
 
+def test_nvml_sample_summary_decodes_reason_bits():
+    t = 1000.0
+    samples = [(t - 1, 1000, 1965, 0x0), (t + 0.001, 1900, 1965, 0x4), (t + 0.003, 1800, 1965, 0x4 | 0x40),
+               (t + 0.005, 1965, 1965, 0x1), (t + 2, 500, 1965, 0x8)]
+    s = bench.ClockSampler.summarize_samples(samples, t, t + 0.01)
+    assert s["samples"] == 3 and s["in_timed_region"] and s["sm_mhz"] == 1900.0
+    assert s["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]   # 0x1 (idle) is not a reason kept
+    s = bench.ClockSampler.summarize_samples(samples, t + 10, t + 11)
+    assert s["samples"] == 5 and not s["in_timed_region"] and "hw_slowdown" in s["reasons"]
+    assert bench.ClockSampler.summarize_samples([]) is None
+
+
 def test_launch_count_follows_the_slide_plan():
     import workloads
     from streaming_video_audio_b200.window import StreamingWindow
