@@ -60,6 +60,10 @@ constexpr int kWarpTma = 12, kWarpMma = 13;
 constexpr int kPanelBytes = 128 * 128;   // 128 rows x 128 bytes (64 bf16), one swizzle-128B panel
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
+// The producer's waits for a free stage are never on the critical path (loads
+// run a stage ahead): it polls with a suspend-time hint, leaving the issue
+// slots of its SM sub-partition to the softmax warps there.
+constexpr uint32_t kProducerSuspend = 5000;
 
 
 // Registers per thread after reallocation (launch: 65536 / 512 = 128 each):
@@ -430,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int st = j % kStages;
                     const uint32_t ph = (j / kStages) & 1;
                     const int row0 = seg_start[w.s] + w.t * kTileN;
-                    if (!mbar_wait(&k_empty[st], ph ^ 1, abort_flag, p.status, limit)) break;
+                    if (!mbar_wait(&k_empty[st], ph ^ 1, abort_flag, p.status, limit, kProducerSuspend)) break;
                     if (j != p.withheld_tile) {
                         mbar_expect_tx(&k_full[st], L::kTileBytes);
 #pragma unroll
@@ -439,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                         &k_full[st]);
                         k_last[st] = j;
                     }
-                    if (!mbar_wait(&v_empty[st], ph ^ 1, abort_flag, p.status, limit)) break;
+                    if (!mbar_wait(&v_empty[st], ph ^ 1, abort_flag, p.status, limit, kProducerSuspend)) break;
                     mbar_expect_tx(&v_full[st], L::kTileBytes);
 #pragma unroll
                     for (int pn = 0; pn < L::kPanels; ++pn)
