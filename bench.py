@@ -4,15 +4,17 @@
                     [--no-graphs] [--no-cpu-baseline] [--row {step,moving,qknorm,window,ulysses}]
 
 A step is one pass of the whole hot path on one batch of synthetic inputs
-resident in HBM: the window slide of the tiered configs (a1: the frames that
-cross a tier boundary are pooled into the older tier and the previous chunk's
-clean frames become the recent ones), KV append of the chunk (a2), RoPE of
-the chunk queries and of every window key (a3) and the fused chunk attention
-(a4).  Default workload: the tiered streaming chunk (config 3), the one
-config on which all four steps run.
+resident in HBM: the window slide of the tiered configs (a1: the stream clock
+advances, the frames that cross a tier boundary are pooled into the older
+tier and the previous chunk's clean frames become the recent ones, each key
+rotated once as it enters its slot), KV append of the chunk with its RoPE
+(a2 + a3), RoPE of the chunk queries and of the prefix keys (a3) and the
+fused chunk attention (a4).  Default workload: the tiered streaming chunk
+(config 3), the one config on which all four steps run.
 
-The step is replayed from CUDA graphs (one pair per ring state, all
-captured during warm-up); --no-graphs launches its kernels one by one.
+The step is replayed from CUDA graphs (one pair per ring state, captured in
+a phase of their own before the warm-up); --no-graphs launches its kernels
+one by one.
 
 Printed: ONE JSON line (rank 0) with attention TFLOP/s of the whole job
 (algorithmic FLOPs 4*Lq*Lkv*D per head over valid tokens only, summed over
