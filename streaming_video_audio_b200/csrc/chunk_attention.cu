@@ -186,7 +186,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    if (threadIdx.x == 0) {
+    if (warp == kWarpTma && lane == 0) {
+        // The producer thread sets the CTA up, and sends the Q loads on their
+        // way before it reads the segment lengths (their latency overlaps).
         mbar_init(q_full, 1);
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&k_full[i], 1);
@@ -202,6 +204,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
+        fence_mbarrier_init();
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+        mbar_expect_tx(q_full, kQTiles * L::kTileBytes);
+#pragma unroll
+        for (int t = 0; t < kQTiles; ++t)
+#pragma unroll
+            for (int pn = 0; pn < L::kPanels; ++pn)
+                tma_load_3d(smem + L::kQ + t * L::kTileBytes + pn * kPanelBytes, &tmQ, pn * 64, q0 + t * kTileM, bh,
+                            q_full);
         int total = 0;
 #pragma unroll
         for (int s = 0; s < SR_MAX_SEG; ++s) {   // static indices keep the param arrays out of local memory
@@ -223,7 +236,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         n_tiles_s[0] = tile1 - tile0;
         walk_start[0] = s0;
         walk_start[1] = k;
-        fence_mbarrier_init();
     }
     if (warp == kWarpMma) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -413,17 +425,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         regs_decrease<kRegOther>();
         if (warp == kWarpTma) {
             // ============================================================ TMA producer
+            // (Q is on its way since the set-up)
+            if (lane == 0 && n_tiles == 0) mbar_drain(q_full, 0, limit);   // no tile: only Q to see land
             if (lane == 0 && n_tiles > 0) {
-                tma_prefetch_desc(&tmQ);
-                tma_prefetch_desc(&tmK);
-                tma_prefetch_desc(&tmV);
-                mbar_expect_tx(q_full, kQTiles * L::kTileBytes);
-#pragma unroll
-                for (int t = 0; t < kQTiles; ++t)
-#pragma unroll
-                    for (int pn = 0; pn < L::kPanels; ++pn)
-                        tma_load_3d(smem + L::kQ + t * L::kTileBytes + pn * kPanelBytes, &tmQ, pn * 64,
-                                    q0 + t * kTileM, bh, q_full);
                 int k_last[kStages], v_last[kStages];   // last tile loaded into each stage (for the drain)
 #pragma unroll
                 for (int i = 0; i < kStages; ++i) k_last[i] = v_last[i] = -1;
