@@ -98,7 +98,7 @@ class ClockSampler:
     """SM clocks and throttle reasons of the timed GPU, sampled while the
     timed region runs; mark() brackets that region on the host clock, and
     stop() keeps the samples taken inside it (all samples, flagged, when none
-    fell inside).  NVML is polled every 2 ms from a thread (a 20-step region
+    fell inside).  NVML is polled every 1 ms from a thread (a 20-step region
     lasts only ~14 ms); without NVML, nvidia-smi samples every 200 ms."""
     FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -127,7 +127,12 @@ class ClockSampler:
                                              pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)))
                     except pynvml.NVMLError:
                         return
-                    time.sleep(0.002)
+                    time.sleep(0.001)
+            # a busy host thread keeps the GIL for up to the switch interval
+            # (5 ms by default): shorten it so the poller runs inside a short
+            # timed region too
+            self.switch = sys.getswitchinterval()
+            sys.setswitchinterval(2e-4)
             self.thread = threading.Thread(target=poll, daemon=True)
             self.thread.start()
         except Exception:
@@ -154,6 +159,7 @@ class ClockSampler:
         if self.thread is not None:
             self.done.set()
             self.thread.join(timeout=5)
+            sys.setswitchinterval(self.switch)
             return self.summarize_samples(self.samples, *self.window)
         if self.p is None:
             return None
@@ -172,7 +178,7 @@ class ClockSampler:
         """The same summary from NVML samples (time, sm MHz, max MHz, reason bits)."""
         rows = [(ts, float(sm), float(mx), {n for n, bit in cls.REASON_BITS.items() if r & bit})
                 for ts, sm, mx, r in samples]
-        return cls._summary(rows, t0, t1, "nvml, 2 ms")
+        return cls._summary(rows, t0, t1, "nvml, 1 ms")
 
     @staticmethod
     def _summary(samples, t0, t1, source):
