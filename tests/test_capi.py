@@ -45,6 +45,10 @@ def test_attention_rejects_bad_arguments_on_host():
     bad = capi.make_layout([100])
     assert call(args(lay=ctypes.byref(bad))) == capi.SR_ERR_INVALID_ARG and "multiple" in _err(lib)
     assert call(args(B=0)) == capi.SR_OK                       # zero work: nothing launched
+    for n_seg in (0, capi.SR_MAX_SEG + 1):                       # segment count outside [1, SR_MAX_SEG]
+        lay_bad = capi.make_layout([128])
+        lay_bad.n_seg = n_seg
+        assert call(args(lay=ctypes.byref(lay_bad))) == capi.SR_ERR_INVALID_ARG and "n_seg" in _err(lib)
     assert call(args(q=16, k=32, v=48, o=72, kl=1, ql=1)) == capi.SR_ERR_INVALID_ARG   # misaligned o
     assert "aligned" in _err(lib)
 

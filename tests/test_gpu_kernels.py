@@ -265,6 +265,9 @@ def _valid_kv(k, v, b, h, caps, lens_b):
     (128, 3, [128, 1024, 256], [[1, 1000, 129], [128, 7, 256], [0, 513, 255]], [129, 256, 255]),
     (64, 2, [256, 256], [[256, 256], [1, 0]], [200, 1]),
     (128, 2, [128, 256], [[128, 200], [64, 9]], [256, 0]),      # a session without queries
+    # the most segments a window may have, empty ones between full and ragged ones
+    (128, 2, [128, 256, 128, 384, 128, 128, 256, 128], [[100, 0, 128, 300, 0, 1, 256, 77]], [300]),
+    (64, 3, [256, 128, 128, 128, 128, 128, 128, 256], [[0, 0, 5, 128, 0, 64, 0, 255]], [130]),
 ])
 def test_attention_matches_oracle(D, H, caps, lens, q_len):
     q, k, v, o, lse = _attention_case(D, H, caps, lens, q_len, seed=20)
