@@ -349,7 +349,8 @@ int sr_set_wait_limit_ns(uint64_t limit_ns);
 
 /* Test hook of that failure path, not for production use (the pages have no
  * counterpart): from the next attention launch on, the load of K tile `tile`
- * (counted from each work item's first tile) is withheld, so the pipeline
+ * (counted from each work item's first tile), and of the V tile that shares
+ * its pipeline stage, is withheld, so the pipeline
  * wait for it runs out after the limit above and the launch reports
  * SR_ERR_DEVICE_TIMEOUT.  Nothing faults or hangs.  -1 (the default) turns it
  * off; < -1 is rejected. */

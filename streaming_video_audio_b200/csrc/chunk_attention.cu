@@ -105,9 +105,9 @@ struct Smem {
     static constexpr int kK = kQ + kQTiles * kTileBytes;
     static constexpr int kV = kK + kStages * kTileBytes;
     static constexpr int kBar = kV + kStages * kTileBytes;
-    // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S],
-    // s_full[2], p_full[2], o_done[2], stats_ready[2], drain
-    static constexpr int kNumBars = 1 + 4 * kStages + 4 * kQTiles + 1;
+    // q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2],
+    // stats_ready[2], drain
+    static constexpr int kNumBars = 1 + 2 * kStages + 4 * kQTiles + 1;
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kRow = kMisc + 16 + 12 * SR_MAX_SEG + 16;   // float l[2][128], m[2][128]
     static constexpr int kEnd = kRow + 2 * kQTiles * kTileM * 4;
@@ -162,11 +162,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBar);
     uint64_t *q_full = bars;
-    uint64_t *k_full = bars + 1;
-    uint64_t *k_empty = k_full + kStages;
-    uint64_t *v_full = k_empty + kStages;
-    uint64_t *v_empty = v_full + kStages;
-    uint64_t *s_full = v_empty + kStages;        // [2] MMA -> softmax t
+    // Stage i % kStages holds K(i) and V(i-1): the two tiles the MMAs of one
+    // period read (PV(i-1) and S(i)), loaded and released under one barrier
+    // pair, so that the issuing thread makes one load wait and one release
+    // commit per KV tile.
+    uint64_t *kv_full = bars + 1;
+    uint64_t *kv_empty = kv_full + kStages;
+    uint64_t *s_full = kv_empty + kStages;       // [2] MMA -> softmax t
     uint64_t *p_full = s_full + kQTiles;         // [2] softmax t -> MMA (P_t written, O_t rescaled)
     uint64_t *o_done = p_full + kQTiles;         // [2] MMA (PV_t) -> epilogue
     uint64_t *stats_ready = o_done + kQTiles;    // [2] softmax t -> epilogue: final row max / sum
@@ -191,10 +193,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // way before it reads the segment lengths (their latency overlaps).
         mbar_init(q_full, 1);
         for (int i = 0; i < kStages; ++i) {
-            mbar_init(&k_full[i], 1);
-            mbar_init(&k_empty[i], 1);
-            mbar_init(&v_full[i], 1);
-            mbar_init(&v_empty[i], 1);
+            mbar_init(&kv_full[i], 1);
+            mbar_init(&kv_empty[i], 1);
         }
         for (int t = 0; t < kQTiles; ++t) {
             mbar_init(&s_full[t], 1);
@@ -428,40 +428,44 @@ __global__ void __launch_bounds__(kThreads, 1)
             // (Q is on its way since the set-up)
             if (lane == 0 && n_tiles == 0) mbar_drain(q_full, 0, limit);   // no tile: only Q to see land
             if (lane == 0 && n_tiles > 0) {
-                int k_last[kStages], v_last[kStages];   // last tile loaded into each stage (for the drain)
+                int kv_last[kStages];   // last stage fill issued into each stage (for the drain)
 #pragma unroll
-                for (int i = 0; i < kStages; ++i) k_last[i] = v_last[i] = -1;
+                for (int i = 0; i < kStages; ++i) kv_last[i] = -1;
                 TileWalk w;
                 w.s = walk_start[0];
                 w.t = walk_start[1];
-                for (int j = 0; j < n_tiles; ++j, w.next(seg_ntile, n_seg)) {
-                    const int st = j % kStages;
-                    const uint32_t ph = (j / kStages) & 1;
-                    const int row0 = seg_start[w.s] + w.t * kTileN;
-                    if (!mbar_wait(&k_empty[st], ph ^ 1, abort_flag, p.status, limit, kProducerSuspend)) break;
-                    if (j != p.withheld_tile) {
-                        mbar_expect_tx(&k_full[st], L::kTileBytes);
+                int row_v = 0;
+                // fill i: K(i) (i < n_tiles) and V(i-1) (i > 0)
+                for (int i = 0; i <= n_tiles; ++i) {
+                    const int st = i % kStages;
+                    const uint32_t ph = (i / kStages) & 1;
+                    const bool has_k = i < n_tiles, has_v = i > 0;
+                    const int row_k = has_k ? seg_start[w.s] + w.t * kTileN : 0;
+                    if (!mbar_wait(&kv_empty[st], ph ^ 1, abort_flag, p.status, limit, kProducerSuspend)) break;
+                    if (!(has_k && i == p.withheld_tile)) {
+                        mbar_expect_tx(&kv_full[st], (has_k && has_v ? 2 : 1) * L::kTileBytes);
+                        if (has_k) {
 #pragma unroll
-                        for (int pn = 0; pn < L::kPanels; ++pn)
-                            tma_load_3d(smem + L::kK + st * L::kTileBytes + pn * kPanelBytes, &tmK, pn * 64, row0, bh,
-                                        &k_full[st]);
-                        k_last[st] = j;
+                            for (int pn = 0; pn < L::kPanels; ++pn)
+                                tma_load_3d(smem + L::kK + st * L::kTileBytes + pn * kPanelBytes, &tmK, pn * 64,
+                                            row_k, bh, &kv_full[st]);
+                        }
+                        if (has_v) {
+#pragma unroll
+                            for (int pn = 0; pn < L::kPanels; ++pn)
+                                tma_load_3d(smem + L::kV + st * L::kTileBytes + pn * kPanelBytes, &tmV, pn * 64,
+                                            row_v, bh, &kv_full[st]);
+                        }
+                        kv_last[st] = i;
                     }
-                    if (!mbar_wait(&v_empty[st], ph ^ 1, abort_flag, p.status, limit, kProducerSuspend)) break;
-                    mbar_expect_tx(&v_full[st], L::kTileBytes);
-#pragma unroll
-                    for (int pn = 0; pn < L::kPanels; ++pn)
-                        tma_load_3d(smem + L::kV + st * L::kTileBytes + pn * kPanelBytes, &tmV, pn * 64, row0, bh,
-                                    &v_full[st]);
-                    v_last[st] = j;
+                    row_v = row_k;
+                    if (has_k) w.next(seg_ntile, n_seg);
                 }
                 if (*abort_flag) {
                     // wait, bounded, for the loads still in flight into this CTA
                     mbar_drain(q_full, 0, limit);
-                    for (int i = 0; i < kStages; ++i) {
-                        if (k_last[i] >= 0) mbar_drain(&k_full[i], (k_last[i] / kStages) & 1, limit);
-                        if (v_last[i] >= 0) mbar_drain(&v_full[i], (v_last[i] / kStages) & 1, limit);
-                    }
+                    for (int i = 0; i < kStages; ++i)
+                        if (kv_last[i] >= 0) mbar_drain(&kv_full[i], (kv_last[i] / kStages) & 1, limit);
                 }
             }
         } else if (warp == kWarpMma) {
@@ -506,30 +510,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                     return true;
                 };
                 bool ok = mbar_wait(q_full, 0, abort_flag, p.status, limit) &&
-                          mbar_wait(&k_full[0], 0, abort_flag, p.status, limit);
+                          mbar_wait(&kv_full[0], 0, abort_flag, p.status, limit);
                 if (ok) {
                     tc_fence_after();
                     issue_qk(0, 0);
                     issue_qk(1, 0);
-                    umma_commit(&k_empty[0]);
+                    umma_commit(&kv_empty[0]);
                 }
                 for (int j = 0; ok && j < n_tiles; ++j) {
-                    const int st = j % kStages;
-                    const int st1 = (j + 1) % kStages;
+                    // stage st holds V(j) and K(j+1)
+                    const int st = (j + 1) % kStages;
                     const bool more = j + 1 < n_tiles;
-                    // load waits first (the tiles landed long ago): once P arrives, the
-                    // MMAs follow each other without a wait that would idle the pipe
-                    if (!(ok = mbar_wait(&v_full[st], (j / kStages) & 1, abort_flag, p.status, limit))) break;
-                    if (more && !(ok = mbar_wait(&k_full[st1], ((j + 1) / kStages) & 1, abort_flag, p.status, limit)))
-                        break;
+                    // the load wait first (the tiles landed long ago): once P arrives,
+                    // the MMAs follow each other without a wait that would idle the pipe
+                    if (!(ok = mbar_wait(&kv_full[st], ((j + 1) / kStages) & 1, abort_flag, p.status, limit))) break;
                     if (!(ok = pv_step(0, st, j, !more))) break;
-                    if (more) issue_qk(0, st1);
+                    if (more) issue_qk(0, st);
                     if (!(ok = pv_step(1, st, j, !more))) break;
-                    umma_commit(&v_empty[st]);
-                    if (more) {
-                        issue_qk(1, st1);
-                        umma_commit(&k_empty[st1]);
-                    }
+                    if (more) issue_qk(1, st);
+                    umma_commit(&kv_empty[st]);
                 }
                 // every MMA issued so far complete before the tensor and shared
                 // memory may be released (matters after an abort)
