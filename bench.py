@@ -98,8 +98,11 @@ class ClockSampler:
     """SM clocks and throttle reasons of the timed GPU, sampled while the
     timed region runs; mark() brackets that region on the host clock, and
     stop() keeps the samples taken inside it (all samples, flagged, when none
-    fell inside).  NVML is polled every 1 ms from a thread (a 20-step region
-    lasts only ~14 ms); without NVML, nvidia-smi samples every 200 ms."""
+    fell inside).  NVML is polled from a thread as fast as it answers (a
+    20-step region lasts only ~14 ms, an NVML query can take a few ms), and
+    await_sample() lets the host, its launches queued, wait until one sample
+    has been taken inside the region while the GPU is still busy with them.
+    Without NVML, nvidia-smi samples every 200 ms."""
     FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -118,16 +121,22 @@ class ClockSampler:
             h = pynvml.nvmlDeviceGetHandleByPciBusId(
                 f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0")
             self.done = threading.Event()
+            self.fresh = threading.Event()   # a sample taken after mark(0)
+            max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
 
             def poll():
                 while not self.done.is_set():
                     try:
-                        self.samples.append((time.time(), pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
-                                             pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM),
-                                             pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)))
+                        a = time.time()
+                        sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                        r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        ts = 0.5 * (a + time.time())   # the readings are of the middle of the queries
                     except pynvml.NVMLError:
                         return
-                    time.sleep(0.001)
+                    self.samples.append((ts, sm, max_mhz, r))
+                    if self.window[0] is not None and a >= self.window[0]:
+                        self.fresh.set()
+                    time.sleep(0.0002)
             # a busy host thread keeps the GIL for up to the switch interval
             # (5 ms by default): shorten it so the poller runs inside a short
             # timed region too
@@ -155,6 +164,12 @@ class ClockSampler:
     def mark(self, i: int) -> None:
         self.window[i] = time.time()
 
+    def await_sample(self, timeout: float = 0.05) -> None:
+        """Block the host (its launches already queued) until the poller has
+        taken a sample inside the timed region, at most `timeout` seconds."""
+        if self.thread is not None:
+            self.fresh.wait(timeout)
+
     def stop(self):
         if self.thread is not None:
             self.done.set()
@@ -178,7 +193,7 @@ class ClockSampler:
         """The same summary from NVML samples (time, sm MHz, max MHz, reason bits)."""
         rows = [(ts, float(sm), float(mx), {n for n, bit in cls.REASON_BITS.items() if r & bit})
                 for ts, sm, mx, r in samples]
-        return cls._summary(rows, t0, t1, "nvml, 1 ms")
+        return cls._summary(rows, t0, t1, "nvml")
 
     @staticmethod
     def _summary(samples, t0, t1, source):
@@ -554,6 +569,7 @@ def _timed(step, K, W, local, dist=None, before=None, capture=0):
     for i in range(K):
         step(W + i, marks[i])
     stop.record(stream)
+    sampler.await_sample()
     torch.cuda.synchronize()
     sampler.mark(1)
     if dist:
@@ -810,6 +826,7 @@ def main():
     for i in range(K):
         one_step(capture_steps + W + i, evs[i])
         bounds[i + 1].record(stream)
+    sampler.await_sample()
     torch.cuda.synchronize()
     sampler.mark(1)
     if dist:

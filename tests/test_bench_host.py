@@ -35,6 +35,22 @@ def test_nvml_sample_summary_decodes_reason_bits():
     assert bench.ClockSampler.summarize_samples([]) is None
 
 
+def test_await_sample_is_bounded():
+    import threading
+    import time
+    s = object.__new__(bench.ClockSampler)
+    s.thread = None
+    s.await_sample(5.0)                       # nvidia-smi fallback: nothing to wait for
+    s.thread, s.fresh = object(), threading.Event()
+    t = time.time()
+    s.await_sample(0.02)                      # no sample comes: gives up after the timeout
+    assert 0.015 <= time.time() - t < 1.0
+    s.fresh.set()
+    t = time.time()
+    s.await_sample(5.0)                       # a sample inside the region: returns at once
+    assert time.time() - t < 0.5
+
+
 def test_launch_count_follows_the_slide_plan():
     import workloads
     from streaming_video_audio_b200.window import StreamingWindow
