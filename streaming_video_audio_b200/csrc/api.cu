@@ -38,8 +38,9 @@ int set_cuda_error(const char *what, cudaError_t e) {
     return set_error(SR_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
 }
 
-int make_tmap_bf16_3d(CUtensorMap *tm, const void *base, uint64_t inner, uint64_t rows, uint64_t outer,
-                      uint32_t box_inner, uint32_t box_rows) {
+namespace {
+// cuTensorMapEncodeTiled from the driver, resolved once (nullptr if absent)
+EncodeTiledFn encode_fn() {
     std::call_once(g_encode_once, [] {
         void *fn = nullptr;
         cudaDriverEntryPointQueryResult q;
@@ -47,14 +48,36 @@ int make_tmap_bf16_3d(CUtensorMap *tm, const void *base, uint64_t inner, uint64_
             q == cudaDriverEntryPointSuccess)
             g_encode = reinterpret_cast<EncodeTiledFn>(fn);
     });
-    if (!g_encode) return set_error(SR_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    return g_encode;
+}
+}  // namespace
+
+int make_tmap_bf16_3d(CUtensorMap *tm, const void *base, uint64_t inner, uint64_t rows, uint64_t outer,
+                      uint32_t box_inner, uint32_t box_rows) {
+    const EncodeTiledFn enc = encode_fn();
+    if (!enc) return set_error(SR_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
     const cuuint64_t dims[3] = {inner, rows, outer};
     const cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
     const cuuint32_t box[3] = {box_inner, box_rows, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
-                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return set_error(SR_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", int(r));
+    return SR_OK;
+}
+
+int make_tmap_bf16_4d(CUtensorMap *tm, void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3,
+                      uint32_t box0, uint32_t box2) {
+    const EncodeTiledFn enc = encode_fn();
+    if (!enc) return set_error(SR_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    const cuuint64_t dims[4] = {d0, d1, d2, d3};
+    const cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};
+    const cuuint32_t box[4] = {box0, 1, box2, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return set_error(SR_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", int(r));
     return SR_OK;
 }

@@ -70,6 +70,12 @@ constexpr uint32_t kProducerSuspend = 5000;
 // 2 x 128 x 160 + 128 x 88 + 128 x 104 = 65536 (the launch total; no spills).
 constexpr int kRegSoftmax = 160, kRegCorrection = 88, kRegOther = 104;
 
+// Byte offset of 16-byte chunk k of row `row` in a tile of 64-column bf16
+// panels (128 rows x 128 bytes each) laid out with the 128-byte swizzle.
+__device__ __forceinline__ int sw128_offset(int row, int k) {
+    return (k >> 3) * kPanelBytes + row * 128 + (((k & 7) ^ (row & 7)) << 4);
+}
+
 __host__ __device__ constexpr uint32_t tmem_s(int t) { return static_cast<uint32_t>(t) * 128u; }
 __host__ __device__ constexpr uint32_t tmem_o(int t) { return 256u + static_cast<uint32_t>(t) * 128u; }
 
@@ -91,7 +97,7 @@ struct AttnParams {
     int32_t qb_per_head;     // 256-row query blocks per (session, head)
     int32_t n_full;
     int32_t split;
-    float *ws_o;             // [slot][2][128][D] unnormalised partial O (log2-domain max m, sum l)
+    float *ws_o;             // [slot][2][D/4][128][4] unnormalised partial O (column blocks of 4)
     float *ws_ml;            // [slot][m | l][2][128]
     uint64_t wait_limit_ns;
     int32_t withheld_tile;   // test hook: the K tile whose load is withheld (-1: none)
@@ -136,7 +142,8 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                           const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                           const AttnParams p) {
     using L = Smem<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -343,6 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp < 4 * kQTiles + 4) {
         // ================================================================ epilogue
         regs_decrease<kRegCorrection>();
+        constexpr int kRowChunks = D / 8;   // 16-byte chunks in one bf16 row of O
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
@@ -353,8 +361,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int t = 0; t < kQTiles; ++t) {
                 const int grow = q0 + t * kTileM + row;
                 const bool row_ok = grow < q_len;
-                __nv_bfloat16 *orow = p.o + ((static_cast<size_t>(b) * p.q_cap + grow) * p.n_heads + h) * D;
                 if (n_tiles == 0) {
+                    __nv_bfloat16 *orow = p.o + ((static_cast<size_t>(b) * p.q_cap + grow) * p.n_heads + h) * D;
                     if (row_ok) {
                         for (int d = 0; d < D; d += 8) *reinterpret_cast<uint4 *>(orow + d) = make_uint4(0, 0, 0, 0);
                         if (p.lse) p.lse[static_cast<size_t>(bh) * p.q_cap + grow] = -INFINITY;
@@ -367,27 +375,60 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const float l_row = row_l[t * kTileM + row];
                 const float inv_l = 1.0f / l_row;
+                // This warp's 32 rows of O_t, normalised and packed to bf16, are
+                // staged in Q_t's shared memory (no MMA reads Q_t once O_t is
+                // final) in the copy engine's 128-byte swizzled layout (64-column
+                // panels, 16-byte chunks XOR-ed with the row: no bank conflicts),
+                // then stored by one tiled copy per panel when all 32 rows are
+                // valid, else by whole-row coalesced stores of the valid rows: a
+                // thread per row would touch 32 lines per store instruction.
+                uint8_t *stage = smem + L::kQ + t * L::kTileBytes;
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t r[32];
                     tmem_ld32(tmem + lane_base + tmem_o(t) + c * 32, r);
                     tmem_wait_ld();
-                    if (row_ok) {
 #pragma unroll
-                        for (int e = 0; e < 32; e += 8) {
-                            uint4 v;
-                            v.x = pack_bf16x2(__uint_as_float(r[e + 0]) * inv_l, __uint_as_float(r[e + 1]) * inv_l);
-                            v.y = pack_bf16x2(__uint_as_float(r[e + 2]) * inv_l, __uint_as_float(r[e + 3]) * inv_l);
-                            v.z = pack_bf16x2(__uint_as_float(r[e + 4]) * inv_l, __uint_as_float(r[e + 5]) * inv_l);
-                            v.w = pack_bf16x2(__uint_as_float(r[e + 6]) * inv_l, __uint_as_float(r[e + 7]) * inv_l);
-                            *reinterpret_cast<uint4 *>(orow + c * 32 + e) = v;
-                        }
+                    for (int e = 0; e < 32; e += 8) {
+                        uint4 v;
+                        v.x = pack_bf16x2(__uint_as_float(r[e + 0]) * inv_l, __uint_as_float(r[e + 1]) * inv_l);
+                        v.y = pack_bf16x2(__uint_as_float(r[e + 2]) * inv_l, __uint_as_float(r[e + 3]) * inv_l);
+                        v.z = pack_bf16x2(__uint_as_float(r[e + 4]) * inv_l, __uint_as_float(r[e + 5]) * inv_l);
+                        v.w = pack_bf16x2(__uint_as_float(r[e + 6]) * inv_l, __uint_as_float(r[e + 7]) * inv_l);
+                        const int k = c * 4 + e / 8;   // 16-byte chunk of the row
+                        *reinterpret_cast<uint4 *>(stage + sw128_offset(row, k)) = v;
+                    }
+                }
+                const int r0 = q0 + t * kTileM + quarter * 32;   // this warp's first row
+                if (r0 + 32 <= q_len) {
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+#pragma unroll
+                        for (int pn = 0; pn < L::kPanels; ++pn)
+                            tma_store_4d(&tmO, stage + pn * kPanelBytes + quarter * 32 * 128, pn * 64, h, r0, b);
+                        bulk_commit_group();
+                    }
+                } else {
+                    __syncwarp();
+                    const int sub = lane / kRowChunks, k = lane % kRowChunks;
+#pragma unroll 4
+                    for (int i = 0; i < 32; i += 32 / kRowChunks) {
+                        const int r = quarter * 32 + i + sub;
+                        const int g = q0 + t * kTileM + r;
+                        const uint4 v = *reinterpret_cast<const uint4 *>(stage + sw128_offset(r, k));
+                        if (g < q_len)
+                            *reinterpret_cast<uint4 *>(
+                                p.o + ((static_cast<size_t>(b) * p.q_cap + g) * p.n_heads + h) * D + k * 8) = v;
                     }
                 }
                 if (row_ok && p.lse)
                     p.lse[static_cast<size_t>(bh) * p.q_cap + grow] =
                         (row_m[t * kTileM + row] + log2f(l_row)) * 0.69314718055994531f;
             }
+            // the tiled stores have read their shared-memory source before the
+            // CTA's shared memory is released
+            if (lane == 0) bulk_wait_group_read0();
         } else {
             // Split unit: publish this part's unnormalised (O, m, l); the
             // combine kernel that follows on the stream merges the parts.
@@ -395,8 +436,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             float *ws_m = p.ws_ml + static_cast<size_t>(slot) * 4 * kTileM;
 #pragma unroll 1
             for (int t = 0; t < kQTiles; ++t) {
-                float *o_part =
-                    p.ws_o + (static_cast<size_t>(slot) * kQTiles + t) * kTileM * D + static_cast<size_t>(row) * D;
+                // column blocks of 4 floats, rows inner: a warp's store is 512
+                // contiguous bytes
+                float *o_part = p.ws_o + (static_cast<size_t>(slot) * kQTiles + t) * kTileM * D + row * 4;
                 float m_part = -INFINITY, l_part = 0.f;
                 if (n_tiles > 0) {
                     if (!ok) break;
@@ -412,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tmem_wait_ld();
 #pragma unroll
                         for (int e = 0; e < 32; e += 4)
-                            __stcg(reinterpret_cast<float4 *>(o_part + c * 32 + e),
+                            __stcg(reinterpret_cast<float4 *>(o_part + (c * 8 + e / 4) * kTileM * 4),
                                    make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
                                                __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3])));
                     }
@@ -549,7 +591,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // Merges the KV parts of every split unit: for each query row,
 //   M = max_q m_q,  L = sum_q l_q 2^(m_q - M),  O = sum_q 2^(m_q - M) O_q / L
-// (O_q unnormalised, m in log2 units).  One thread per (unit, row, 8 columns).
+// (O_q unnormalised, m in log2 units).  One thread per (unit, row, 8 columns);
+// a warp takes 8 rows x 4 column chunks, so that its reads of the partials
+// (column blocks, rows inner) and its writes of O (rows, columns inner) both
+// cover whole runs of 64 to 128 bytes.
 struct CombineParams {
     const float *ws_o;
     const float *ws_ml;
@@ -565,9 +610,12 @@ __global__ void __launch_bounds__(256) split_combine_kernel(const CombineParams 
     const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     const int64_t total = static_cast<int64_t>(c.tail_units) * kQTiles * kTileM * kChunks;
     if (idx >= total) return;
-    const int chunk = static_cast<int>(idx % kChunks);
-    const int r2 = static_cast<int>((idx / kChunks) % (kQTiles * kTileM));   // row within the 256-row block
-    const int tail = static_cast<int>(idx / (kChunks * kQTiles * kTileM));
+    static_assert(kChunks % 4 == 0, "4 column chunks per warp");
+    const int lane = static_cast<int>(idx & 31);
+    const int64_t wg = idx >> 5;   // (tail, 8-row block, 4-chunk block), chunk blocks fastest
+    const int r2 = static_cast<int>((wg / (kChunks / 4)) % (kQTiles * kTileM / 8)) * 8 + (lane & 7);   // row in the 256-row block
+    const int chunk = static_cast<int>(wg % (kChunks / 4)) * 4 + (lane >> 3);
+    const int tail = static_cast<int>(wg / ((kChunks / 4) * (kQTiles * kTileM / 8)));
     const int t = r2 / kTileM, row = r2 % kTileM;
     const int unit = c.n_full + tail;
     const int qb = unit % c.qb_per_head, bh = unit / c.qb_per_head;
@@ -584,10 +632,10 @@ __global__ void __launch_bounds__(256) split_combine_kernel(const CombineParams 
         if (!(lq > 0.f)) continue;
         const float w = fast_exp2(mq[t * kTileM + row] - mmax);
         lsum += lq * w;
-        const float *oq =
-            c.ws_o + (static_cast<size_t>(tail * c.split + q) * kQTiles + t) * kTileM * D + static_cast<size_t>(row) * D + chunk * 8;
+        const float *oq = c.ws_o + (static_cast<size_t>(tail * c.split + q) * kQTiles + t) * kTileM * D +
+                          (2 * chunk * kTileM + row) * 4;
         const float4 x0 = *reinterpret_cast<const float4 *>(oq);
-        const float4 x1 = *reinterpret_cast<const float4 *>(oq + 4);
+        const float4 x1 = *reinterpret_cast<const float4 *>(oq + kTileM * 4);
         acc[0] += w * x0.x; acc[1] += w * x0.y; acc[2] += w * x0.z; acc[3] += w * x0.w;
         acc[4] += w * x1.x; acc[5] += w * x1.y; acc[6] += w * x1.z; acc[7] += w * x1.w;
     }
@@ -618,11 +666,15 @@ int sm_count() {
 template <int D>
 int launch(const AttnLaunch &a) {
     using L = Smem<D>;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     const uint64_t bh = static_cast<uint64_t>(a.n_batch) * a.n_heads;
     int rc = make_tmap_bf16_3d(&tq, a.q, D, static_cast<uint64_t>(a.q_cap), bh, 64, kTileM);
     if (rc == SR_OK) rc = make_tmap_bf16_3d(&tk, a.k, D, static_cast<uint64_t>(a.kv_tokens), bh, 64, kTileN);
     if (rc == SR_OK) rc = make_tmap_bf16_3d(&tv, a.v, D, static_cast<uint64_t>(a.kv_tokens), bh, 64, kTileN);
+    // o [n_batch][q_cap][n_heads][D], stored in boxes of 32 rows x 64 columns
+    if (rc == SR_OK)
+        rc = make_tmap_bf16_4d(&to, a.o, D, static_cast<uint64_t>(a.n_heads), static_cast<uint64_t>(a.q_cap),
+                               static_cast<uint64_t>(a.n_batch), 64, 32);
     if (rc != SR_OK) return rc;
     AttnParams p{};
     p.o = static_cast<__nv_bfloat16 *>(a.o);
@@ -666,7 +718,7 @@ int launch(const AttnLaunch &a) {
         if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
     if (items > 0x7fffffff) return set_error(SR_ERR_INVALID_ARG, "chunk_attention: too many work items");
-    chunk_attention_kernel<D><<<static_cast<unsigned>(items), kThreads, L::kAlloc, a.stream>>>(tq, tk, tv, p);
+    chunk_attention_kernel<D><<<static_cast<unsigned>(items), kThreads, L::kAlloc, a.stream>>>(tq, tk, tv, to, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return set_cuda_error("chunk_attention launch", e);
     if (p.split > 1)

@@ -18,6 +18,11 @@ int set_cuda_error(const char *what, cudaError_t e);
 int make_tmap_bf16_3d(CUtensorMap *tm, const void *base, uint64_t inner, uint64_t rows, uint64_t outer,
                       uint32_t box_inner, uint32_t box_rows);
 
+// 4-D bf16 tensor map over a dense [d3][d2][d1][d0] tensor (d0 contiguous),
+// box {box0, 1, box2, 1}, 128-byte swizzle (used for tiled stores).
+int make_tmap_bf16_4d(CUtensorMap *tm, void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3,
+                      uint32_t box0, uint32_t box2);
+
 struct AttnLaunch {
     const void *q, *k, *v;
     void *o;
