@@ -304,14 +304,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int c = 0; c < kTileN; ++c) s[c] = c < valid ? s[c] : -INFINITY;
             }
-            // row max over eight independent chains, then a tree
+            // row max over eight independent chains, then a tree: scores 0-7
+            // start the chains, 8-119 join them in pairs of eights, 120-127 alone
             float mx8[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) mx8[i] = s[i];
 #pragma unroll
-            for (int c = 8; c < kTileN; c += 16)
+            for (int c = 8; c + 16 <= kTileN; c += 16)
 #pragma unroll
                 for (int i = 0; i < 8; ++i) mx8[i] = fmax3(mx8[i], s[c + i], s[c + 8 + i]);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mx8[i] = fmaxf(mx8[i], s[kTileN - 8 + i]);
             const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                    fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
             const float m_new = fmaxf(m_run, mx * sl2);
