@@ -439,7 +439,7 @@ constexpr int kGatherHeads = 8;   // head rows a thread keeps in flight
 // cache write and the RoPE in one pass), the token's (cos, sin) pairs
 // computed once for all its heads.
 template <int D, bool kRope>
-__global__ void __launch_bounds__(256) gather_kernel(const GatherArgs a, const RopeTable tab) {
+__global__ void __launch_bounds__(256, 4) gather_kernel(const GatherArgs a, const RopeTable tab) {
     constexpr int kChunks = D / 8;
     __shared__ double s_theta[kRope ? D / 2 : 1];
     if constexpr (kRope) {
