@@ -24,10 +24,12 @@
 //               row in TMEM itself: S_t(j) is issued after PV_t(j-1) and its
 //               commit tracks every earlier MMA, so once S_t(j) has landed
 //               PV_t(j-1) has too, and PV_t(j) waits for this warp's P.
-//   warps 8-11  epilogue: O / l -> bf16 token-major output and LSE (or the
+//   warps 8-11  epilogue: O / l -> bf16 token-major output and LSE, staged in
+//               Q_t's shared memory and stored by tiled copies (or the
 //               unnormalised partials of a split unit).
 //   warp 12     TMA producer: Q0, Q1 once, then K and V tiles (128 tokens) into
-//               two-stage rings, walking only the segments' valid tiles.
+//               a two-stage ring (stage i: K(i) and V(i-1), one barrier pair),
+//               walking only the segments' valid tiles.
 //   warp 13     TMEM owner + single-thread tcgen05.mma issuer, ping-pong order
 //                 PV0(j), S0(j+1) = Q0 K(j+1)^T, PV1(j), S1(j+1)
 //               so the tensor core works on one tile while the other tile's
