@@ -131,3 +131,34 @@ def test_failure_settings_validate_on_host():
     assert lib.sr_set_withheld_kv_tile(-2) == capi.SR_ERR_INVALID_ARG
     assert lib.sr_set_withheld_kv_tile(-1) == capi.SR_OK
     assert lib.sr_set_wait_limit_ns(0) == capi.SR_OK       # back to the default
+
+
+def _device_sms():
+    """SMs of CUDA device 0, or the 148 of a B200 the library assumes without one."""
+    import torch
+    if torch.cuda.is_available():
+        return torch.cuda.get_device_properties(0).multi_processor_count
+    return 148
+
+
+@pytest.mark.parametrize("B,H,D,q_cap", [
+    (1, 40, 128, 3044),   # streaming chunk: 480 units = 3 waves + 36, split 4 ways
+    (1, 40, 128, 2276),   # 360 units = 2 waves + 64, split 2 ways
+    (77, 4, 128, 512),    # VAE window layer: 616 units = 4 waves + 24, split 6 ways
+    (1, 40, 64, 3044),
+    (2, 2, 64, 70),       # 4 units: split 8 ways (the cap)
+    (1, 37, 128, 1024),   # 148 units: whole waves, no workspace
+    (1, 62, 128, 1024),   # 248 units: a remainder of 100 cannot be split in 2
+])
+def test_attention_workspace_follows_the_split_schedule(B, H, D, q_cap):
+    """The split-KV schedule, restated: units are (session, head, 256-row
+    query block); whole waves of one unit per SM run whole; the r units of a
+    last partial wave are split into s = min(8, SMs // r) KV parts when s >= 2.
+    Every part keeps fp32 O for 256 rows x D and (m, l) for 256 rows."""
+    sms = _device_sms()
+    units = B * H * -(-q_cap // 256)
+    rest = units % sms
+    s = min(8, sms // rest) if rest else 0
+    parts = rest * s if s >= 2 else 0
+    expected = parts * 256 * D * 4 + parts * 4 * 128 * 4
+    assert capi.sr_chunk_attention_workspace_bytes(B, H, D, q_cap) == expected
